@@ -1,0 +1,268 @@
+// Log-sum-exp merge of per-slot partials, and the query-stationary decode kernels.
+#pragma once
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace msa {
+
+// ------------------------------------------------------------------------------------
+// Merge: o[i, h] = sum_s exp(lse_s - L) * O_s, L = logsumexp_s lse_s, over the valid
+// slots of (i, g = h / R) in ascending slot order (deterministic). The partial O_s is
+// already normalised by its own softmax sum, so this is the exact softmax over the
+// union of the selected blocks (a fixed-order fp32 reduction; no atomics).
+// ------------------------------------------------------------------------------------
+struct MergeParams {
+  const __nv_bfloat16* opart;  // [rows][G][k][R][D]
+  const float* lse;            // [rows][G][k][R]
+  const int32_t* block_ids;    // [rows0 + rows][G][k] (absolute row index)
+  __nv_bfloat16* o;            // [rows0 + rows][Hq][D]
+  int64_t row0, rows;
+  int G, R, k;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams P) {
+  constexpr int LPH = D / 8;          // lanes per head row (16 bytes each)
+  constexpr int HPW = 32 / LPH;       // head rows per warp
+  const int64_t gw = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int64_t hh = gw * HPW + lane / LPH;
+  const int c = lane % LPH;
+  if (hh >= P.rows * P.G * P.R) return;
+  const int r = static_cast<int>(hh % P.R);
+  const int g = static_cast<int>((hh / P.R) % P.G);
+  const int64_t il = hh / (static_cast<int64_t>(P.R) * P.G);
+  const int64_t i = P.row0 + il;
+  const int32_t* ids = P.block_ids + (i * P.G + g) * P.k;
+  int nv = 0;
+  while (nv < P.k && ids[nv] >= 0) ++nv;
+  const int64_t slot0 = (il * P.G + g) * P.k;
+  float L = -INFINITY;
+  for (int s = 0; s < nv; ++s) L = fmaxf(L, P.lse[(slot0 + s) * P.R + r]);
+  float acc[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
+  float W = 0.0f;
+  for (int s = 0; s < nv; ++s) {
+    const float w = __expf(P.lse[(slot0 + s) * P.R + r] - L);
+    W += w;
+    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(P.opart + ((slot0 + s) * P.R + r) * D) + c);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float2 f = __bfloat1622float2(h2[u]);
+      acc[2 * u] = fmaf(w, f.x, acc[2 * u]);
+      acc[2 * u + 1] = fmaf(w, f.y, acc[2 * u + 1]);
+    }
+  }
+  const float inv = (W > 0.0f) ? 1.0f / W : 0.0f;
+  uint4 out;
+  out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  const int Hq = P.G * P.R;
+  reinterpret_cast<uint4*>(P.o + (i * Hq + g * P.R + r) * D)[c] = out;
+}
+
+// ------------------------------------------------------------------------------------
+// Decode, Index Branch: block maxima of the one new query per sequence against every
+// full block before its local block (query-stationary: the index-key cache streams
+// through once, 64 contiguous bytes per lane per load).
+// ------------------------------------------------------------------------------------
+struct DecodeScanParams {
+  const __nv_bfloat16* q_idx;   // [B][G][DI]
+  const __nv_bfloat16* k_idx;   // [B][Lmax][G][DI]
+  const int32_t* seqlens;
+  uint32_t* maxima;             // [B][G][nbmax]
+  int B, G, nbmax;
+  int64_t Lmax;
+};
+
+// grid (nbmax, B), 256 threads: one CTA per (sequence, block). Needs G * DI / 32 to be
+// a power of two <= 32 (checked by the host).
+template <int DI>
+__global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant__ DecodeScanParams P) {
+  __shared__ uint32_t smax[32];
+  const int b = blockIdx.y, kb = blockIdx.x;
+  const int L = P.seqlens[b];
+  if (L < 1 || L > P.Lmax) {
+    if (kb == 0 && threadIdx.x == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidDecodeScan);
+    return;
+  }
+  const int bl = (L - 1) / 128;
+  if (kb >= bl) return;
+  const int cpt = P.G * DI / 32;             // 64-byte chunks per token
+  constexpr int LPG = DI / 32;               // lanes (chunks) per group
+  const int lane = threadIdx.x & 31;
+  const int w = lane % cpt;                  // constant per lane since cpt | 32
+  const int g = w / LPG;
+  const int qoff = (w % LPG) * 32;
+  if (threadIdx.x < 32) smax[threadIdx.x] = 0u;
+  float qv[32];
+  {
+    const uint4* qp = reinterpret_cast<const uint4*>(P.q_idx + (static_cast<int64_t>(b) * P.G + g) * DI + qoff);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 raw = __ldg(qp + u);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(h2[t]);
+        qv[u * 8 + 2 * t] = f.x;
+        qv[u * 8 + 2 * t + 1] = f.y;
+      }
+    }
+  }
+  __syncthreads();
+  const uint4* base = reinterpret_cast<const uint4*>(P.k_idx + (static_cast<int64_t>(b) * P.Lmax + kb * 128) *
+                                                                   P.G * DI);
+  const int nchunks = 128 * cpt;
+  float best = -INFINITY;
+  for (int c0 = threadIdx.x; c0 < nchunks; c0 += 256 * 2) {
+    uint4 raw[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + h * 256;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) raw[h][u] = (c < nchunks) ? __ldg(base + static_cast<int64_t>(c) * 4 + u) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[h][u]);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(h2[t]);
+          acc = fmaf(qv[u * 8 + 2 * t], f.x, acc);
+          acc = fmaf(qv[u * 8 + 2 * t + 1], f.y, acc);
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < LPG; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (c0 + h * 256 < nchunks) best = fmaxf(best, acc);
+    }
+  }
+  if ((lane % LPG) == 0) {
+    float m = __fadd_rn(best, 0.0f);
+    uint32_t u = __float_as_uint(m);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    atomicMax(&smax[g], u);
+  }
+  __syncthreads();
+  if (threadIdx.x < P.G) P.maxima[(static_cast<int64_t>(b) * P.G + threadIdx.x) * P.nbmax + kb] = smax[threadIdx.x];
+}
+
+// ------------------------------------------------------------------------------------
+// Decode, Main Branch: one CTA per (sequence, group, slot): exact softmax attention of
+// the group's R heads over the slot's block (causal in the local block), written as a
+// normalised partial + lse for the merge kernel.
+// ------------------------------------------------------------------------------------
+struct DecodeAttnParams {
+  const __nv_bfloat16* q;       // [B][Hq][D]
+  const __nv_bfloat16* kc;      // [B][Lmax][G][D]
+  const __nv_bfloat16* vc;
+  const int32_t* seqlens;
+  const int32_t* block_ids;     // [B][G][k]
+  __nv_bfloat16* opart;         // [B][G][k][R][D]
+  float* lse;                   // [B][G][k][R]
+  int B, G, R, k;
+  int64_t Lmax;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant__ DecodeAttnParams P) {
+  constexpr int KS = D + 8;    // padded smem row (bank spread)
+  extern __shared__ uint8_t dsm[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(dsm);
+  __nv_bfloat16* Vs = Ks + 128 * KS;
+  float* Qs = reinterpret_cast<float*>(Vs + 128 * KS);   // [R][D]
+  float* Ss = Qs + P.R * D;                              // [R][128]
+  float* stat = Ss + P.R * 128;                          // [R][2]: max, 1/sum
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int blk = P.block_ids[(static_cast<int64_t>(b) * P.G + g) * P.k + s];
+  if (blk < 0) return;
+  const int L = P.seqlens[b];
+  const int pos = L - 1;
+  if (L < 1 || L > P.Lmax || blk > pos / 128) {
+    if (threadIdx.x == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidDecodeAttn);
+    return;
+  }
+  const int j0 = blk * 128;
+  const int nvalid = min(128, pos - j0 + 1);
+  const int tid = threadIdx.x;
+  // q rows, pre-scaled into log2 units
+  for (int e = tid; e < P.R * D; e += 128) {
+    const int r = e / D, dd = e % D;
+    Qs[e] = __bfloat162float(P.q[(static_cast<int64_t>(b) * P.G * P.R + g * P.R + r) * D + dd]) * P.scale_log2;
+  }
+  // K / V rows of the block (16-byte chunks)
+  constexpr int CPR = D / 8;
+  for (int e = tid; e < 128 * CPR; e += 128) {
+    const int j = e / CPR, c = e % CPR;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (j < nvalid) {
+      const int64_t off = ((static_cast<int64_t>(b) * P.Lmax + j0 + j) * P.G + g) * D;
+      kv = __ldg(reinterpret_cast<const uint4*>(P.kc + off) + c);
+      vv = __ldg(reinterpret_cast<const uint4*>(P.vc + off) + c);
+    }
+    *reinterpret_cast<uint4*>(Ks + j * KS + c * 8) = kv;
+    *reinterpret_cast<uint4*>(Vs + j * KS + c * 8) = vv;
+  }
+  __syncthreads();
+  // scores: thread = key
+  {
+    const int j = tid;
+    for (int r = 0; r < P.R; ++r) {
+      float acc = 0.0f;
+      if (j < nvalid) {
+#pragma unroll 4
+        for (int c = 0; c < CPR; ++c) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(Ks + j * KS + c * 8);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(h2[t]);
+            acc = fmaf(Qs[r * D + c * 8 + 2 * t], f.x, acc);
+            acc = fmaf(Qs[r * D + c * 8 + 2 * t + 1], f.y, acc);
+          }
+        }
+      }
+      Ss[r * 128 + j] = (j < nvalid) ? acc : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // softmax per head: warp w takes heads w, w + 4, ...
+  {
+    const int w = tid >> 5, lane = tid & 31;
+    for (int r = w; r < P.R; r += 4) {
+      float v4[4];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { v4[u] = Ss[r * 128 + lane + 32 * u]; mx = fmaxf(mx, v4[u]); }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { v4[u] = exp2f(v4[u] - mx); sum += v4[u]; Ss[r * 128 + lane + 32 * u] = v4[u]; }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) { stat[2 * r] = mx; stat[2 * r + 1] = sum; }
+    }
+  }
+  __syncthreads();
+  const int64_t slot = (static_cast<int64_t>(b) * P.G + g) * P.k + s;
+  for (int e = tid; e < P.R * D; e += 128) {
+    const int r = e / D, dd = e % D;
+    float acc = 0.0f;
+    for (int j = 0; j < nvalid; ++j) acc = fmaf(Ss[r * 128 + j], __bfloat162float(Vs[j * KS + dd]), acc);
+    P.opart[(slot * P.R + r) * D + dd] = __float2bfloat16_rn(acc / stat[2 * r + 1]);
+  }
+  if (tid < P.R) P.lse[slot * P.R + tid] = (stat[2 * tid] + __log2f(stat[2 * tid + 1])) * 0.69314718055994531f;
+}
+
+}  // namespace msa

@@ -1,0 +1,719 @@
+// C ABI of the MSA library: argument validation, workspace layout, TMA descriptors and
+// the launch sequence of every entry point declared in include/msa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/msa.h"
+#include "common.cuh"
+#include "csr.cuh"
+#include "index_blockmax.cuh"
+#include "kvouter.cuh"
+#include "merge_decode.cuh"
+#include "topk.cuh"
+
+using namespace msa;
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+msa_status_t fail(msa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define MSA_CHECK_CUDA(expr)                                                                     \
+  do {                                                                                           \
+    cudaError_t e_ = (expr);                                                                     \
+    if (e_ != cudaSuccess) return fail(MSA_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define MSA_CHECK_LAUNCH()                                                                        \
+  do {                                                                                            \
+    cudaError_t e_ = cudaGetLastError();                                                          \
+    if (e_ != cudaSuccess) return fail(MSA_ERR_CUDA, "launch failed: %s", cudaGetErrorString(e_)); \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Sub-allocation of the caller's workspace (sizes only when base == nullptr).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carver(void* b) : base(static_cast<uint8_t*>(b)) {}
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off = align_up(off + bytes);
+    return p;
+  }
+};
+
+// ------------------------------- limits / policy -------------------------------
+constexpr int64_t kMaxN = (int64_t(1) << 26) - 1;
+// Maxima buffer of one index launch (bytes). The index branch is cut into query-block
+// ranges whose packed block maxima fit this cap.
+constexpr size_t kMaximaCap = size_t(4) << 30;
+constexpr int64_t kDefaultQueryChunk = 16384;
+
+int64_t tri(int64_t x) { return x * (x - 1) / 2; }
+
+size_t maxima_bytes(int64_t qb0, int64_t qb1, int G) { return size_t(4) * G * 128 * size_t(tri(qb1) - tri(qb0)); }
+
+// [qb0, qb1) ranges of the index branch
+std::vector<std::pair<int, int>> index_chunks(int64_t nb, int G) {
+  std::vector<std::pair<int, int>> out;
+  int64_t qb0 = 0;
+  while (qb0 < nb) {
+    int64_t qb1 = qb0 + 1;
+    // grow while within the cap and within the run table
+    int64_t lo = qb0 + 1, hi = nb;
+    while (lo < hi) {
+      const int64_t mid = (lo + hi + 1) / 2;
+      if (maxima_bytes(qb0, mid, G) <= kMaximaCap && (mid + kIdxKbRun - 1) / kIdxKbRun <= kIdxMaxRuns) lo = mid;
+      else hi = mid - 1;
+    }
+    qb1 = lo;
+    out.emplace_back(int(qb0), int(qb1));
+    qb0 = qb1;
+  }
+  return out;
+}
+
+bool supported_r(int R) { return R == 1 || R == 2 || R == 4 || R == 8 || R == 16; }
+
+msa_status_t check_common(int64_t n, int32_t g, int32_t bk, int32_t k) {
+  if (n < 1 || n > kMaxN) return fail(MSA_ERR_INVALID_ARG, "n=%lld out of range [1, %lld]", (long long)n, (long long)kMaxN);
+  if (g < 1 || g > 64) return fail(MSA_ERR_INVALID_ARG, "g=%d out of range [1, 64]", g);
+  if (k < 1 || k > 32) return fail(MSA_ERR_UNSUPPORTED, "k=%d unsupported (1..32)", k);
+  if (bk != 128) return fail(MSA_ERR_UNSUPPORTED, "bk=%d unsupported (only 128)", bk);
+  return MSA_OK;
+}
+
+msa_status_t check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(MSA_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0) return fail(MSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return MSA_OK;
+}
+
+// ------------------------------- TMA descriptors -------------------------------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map: dims {d0, d1, d2} (d0 innermost), byte strides of dims 1 and 2.
+msa_status_t make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1,
+                         uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {s1, s2};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  const cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return MSA_OK;
+}
+
+int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+template <typename K>
+msa_status_t set_smem(K kernel, int bytes) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "cudaFuncSetAttribute(smem=%d): %s", bytes, cudaGetErrorString(e));
+  return MSA_OK;
+}
+
+// ------------------------------- index branch -------------------------------
+struct IndexLayout {
+  uint32_t* maxima = nullptr;
+  size_t bytes = 0;
+};
+
+IndexLayout index_layout(void* ws, int64_t n, int32_t g) {
+  const int64_t nb = (n + 127) / 128;
+  size_t mx = 0;
+  for (auto& c : index_chunks(nb, g)) mx = std::max(mx, maxima_bytes(c.first, c.second, g));
+  Carver cv(ws);
+  IndexLayout L;
+  L.maxima = static_cast<uint32_t*>(cv.take(std::max<size_t>(mx, 16)));
+  L.bytes = cv.off;
+  return L;
+}
+
+template <int KM>
+void launch_topk_prefill(const TopkPrefillParams& tp, dim3 grid, cudaStream_t st) {
+  topk_prefill_kernel<KM><<<grid, 128, 0, st>>>(tp);
+}
+
+msa_status_t dispatch_topk_prefill(int k, const TopkPrefillParams& tp, dim3 grid, cudaStream_t st) {
+  switch (k - 1) {
+#define MSA_TOPK_CASE(KM) \
+  case KM:                \
+    launch_topk_prefill<KM>(tp, grid, st); break;
+    MSA_TOPK_CASE(0) MSA_TOPK_CASE(1) MSA_TOPK_CASE(2) MSA_TOPK_CASE(3) MSA_TOPK_CASE(4) MSA_TOPK_CASE(5)
+    MSA_TOPK_CASE(6) MSA_TOPK_CASE(7) MSA_TOPK_CASE(8) MSA_TOPK_CASE(9) MSA_TOPK_CASE(10) MSA_TOPK_CASE(11)
+    MSA_TOPK_CASE(12) MSA_TOPK_CASE(13) MSA_TOPK_CASE(14) MSA_TOPK_CASE(15) MSA_TOPK_CASE(16) MSA_TOPK_CASE(17)
+    MSA_TOPK_CASE(18) MSA_TOPK_CASE(19) MSA_TOPK_CASE(20) MSA_TOPK_CASE(21) MSA_TOPK_CASE(22) MSA_TOPK_CASE(23)
+    MSA_TOPK_CASE(24) MSA_TOPK_CASE(25) MSA_TOPK_CASE(26) MSA_TOPK_CASE(27) MSA_TOPK_CASE(28) MSA_TOPK_CASE(29)
+    MSA_TOPK_CASE(30) MSA_TOPK_CASE(31)
+#undef MSA_TOPK_CASE
+    default:
+      return fail(MSA_ERR_UNSUPPORTED, "k=%d", k);
+  }
+  return MSA_OK;
+}
+
+template <int KM>
+void launch_topk_decode(const TopkDecodeParams& tp, cudaStream_t st) {
+  const int rows = tp.B * tp.G;
+  topk_decode_kernel<KM><<<(rows + 127) / 128, 128, 0, st>>>(tp);
+}
+
+msa_status_t dispatch_topk_decode(int k, const TopkDecodeParams& tp, cudaStream_t st) {
+  switch (k - 1) {
+#define MSA_TOPK_CASE(KM) \
+  case KM:                \
+    launch_topk_decode<KM>(tp, st); break;
+    MSA_TOPK_CASE(0) MSA_TOPK_CASE(1) MSA_TOPK_CASE(2) MSA_TOPK_CASE(3) MSA_TOPK_CASE(4) MSA_TOPK_CASE(5)
+    MSA_TOPK_CASE(6) MSA_TOPK_CASE(7) MSA_TOPK_CASE(8) MSA_TOPK_CASE(9) MSA_TOPK_CASE(10) MSA_TOPK_CASE(11)
+    MSA_TOPK_CASE(12) MSA_TOPK_CASE(13) MSA_TOPK_CASE(14) MSA_TOPK_CASE(15) MSA_TOPK_CASE(16) MSA_TOPK_CASE(17)
+    MSA_TOPK_CASE(18) MSA_TOPK_CASE(19) MSA_TOPK_CASE(20) MSA_TOPK_CASE(21) MSA_TOPK_CASE(22) MSA_TOPK_CASE(23)
+    MSA_TOPK_CASE(24) MSA_TOPK_CASE(25) MSA_TOPK_CASE(26) MSA_TOPK_CASE(27) MSA_TOPK_CASE(28) MSA_TOPK_CASE(29)
+    MSA_TOPK_CASE(30) MSA_TOPK_CASE(31)
+#undef MSA_TOPK_CASE
+    default:
+      return fail(MSA_ERR_UNSUPPORTED, "k=%d", k);
+  }
+  return MSA_OK;
+}
+
+template <int DI>
+msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32_t g, const IndexLayout& L,
+                          int32_t* block_ids, int32_t k, cudaStream_t st) {
+  using C = IdxCfg<DI>;
+  static std::once_flag once;
+  static msa_status_t attr = MSA_OK;
+  std::call_once(once, [] { attr = set_smem(index_blockmax_kernel<DI>, C::kSmemBytes); });
+  if (attr != MSA_OK) return attr;
+  const int64_t nb = (n + 127) / 128;
+  const uint64_t row_stride = uint64_t(g) * DI * 2;
+  CUtensorMap tq, tk;
+  const uint32_t box0 = C::kSw64 ? 32 : 64;
+  const CUtensorMapSwizzle sw = C::kSw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  msa_status_t s;
+  if ((s = make_map_3d(&tq, q_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
+  if ((s = make_map_3d(&tk, k_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
+  const int sms = num_sms();
+  for (auto& ch : index_chunks(nb, g)) {
+    const int qb0 = ch.first, qb1 = ch.second;
+    IdxParams P{};
+    P.qb0 = qb0;
+    P.qb1 = qb1;
+    P.npairs = (qb1 - qb0 + 1) / 2;
+    P.G = g;
+    P.maxima = L.maxima;
+    P.region_per_group = 128 * (tri(qb1) - tri(qb0));
+    IdxRunTable T{};
+    // kbend(p) = qa + 1 with a partner tile, qa without; nondecreasing in p
+    auto kbend = [&](int p) { const int qa = qb0 + 2 * p; return (qa + 1 < qb1) ? qa + 1 : qa; };
+    const int maxend = P.npairs > 0 ? kbend(P.npairs - 1) : 0;
+    P.nruns = (maxend + kIdxKbRun - 1) / kIdxKbRun;
+    int acc = 0;
+    for (int c = 0; c < P.nruns; ++c) {
+      int p = 0;
+      while (p < P.npairs && kbend(p) <= c * kIdxKbRun) ++p;
+      T.pmin[c] = p;
+      T.prefix[c] = acc;
+      acc += P.npairs - p;
+    }
+    T.prefix[P.nruns] = acc;
+    P.items_per_group = acc;
+    const int64_t total = int64_t(acc) * g;
+    if (total > 0) {
+      const int grid = int(std::min<int64_t>(sms, total));
+      index_blockmax_kernel<DI><<<grid, kIdxThreads, C::kSmemBytes, st>>>(tq, tk, P, T);
+      MSA_CHECK_LAUNCH();
+    }
+    TopkPrefillParams tp{};
+    tp.maxima = L.maxima;
+    tp.block_ids = block_ids;
+    tp.N = n;
+    tp.G = g;
+    tp.k = k;
+    tp.qb0 = qb0;
+    tp.region_per_group = P.region_per_group;
+    if ((s = dispatch_topk_prefill(k, tp, dim3(qb1 - qb0, g), st)) != MSA_OK) return s;
+    MSA_CHECK_LAUNCH();
+  }
+  return MSA_OK;
+}
+
+msa_status_t run_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx, int32_t k,
+                              int32_t* block_ids, void* ws, cudaStream_t st) {
+  IndexLayout L = index_layout(ws, n, g);
+  switch (d_idx) {
+    case 32: return launch_index<32>(q_idx, k_idx, n, g, L, block_ids, k, st);
+    case 64: return launch_index<64>(q_idx, k_idx, n, g, L, block_ids, k, st);
+    case 128: return launch_index<128>(q_idx, k_idx, n, g, L, block_ids, k, st);
+    default: return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d", d_idx);
+  }
+}
+
+// ------------------------------- main branch (prefill) -------------------------------
+struct AttnLayout {
+  int64_t chunk_blocks = 0;   // query blocks per chunk
+  uint32_t *hist = nullptr, *totals = nullptr, *bstart = nullptr, *istart = nullptr;
+  int32_t* entries = nullptr;
+  int4* items = nullptr;
+  void* opart = nullptr;
+  float* lse = nullptr;
+  size_t bytes = 0;
+};
+
+int rows_per_query(int R) { return R < 8 ? 8 : R; }
+
+AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, int32_t k, int64_t query_chunk) {
+  const int64_t nb = (n + 127) / 128;
+  const int R = hq / g;
+  const int TQ = 128 / rows_per_query(R);
+  int64_t cq = (query_chunk > 0 ? query_chunk : kDefaultQueryChunk) / 128;
+  cq = std::max<int64_t>(1, std::min(cq, nb));
+  AttnLayout L;
+  L.chunk_blocks = cq;
+  const int64_t rows = cq * 128;
+  const int64_t nbuck = int64_t(g) * nb;
+  const int64_t max_entries = rows * g * k;
+  const int64_t max_items = max_entries / (int64_t(TQ) * kKvItemTiles) + nbuck + 1;
+  Carver cv(ws);
+  L.hist = static_cast<uint32_t*>(cv.take(size_t(nbuck) * cq * 4));
+  L.totals = static_cast<uint32_t*>(cv.take(size_t(nbuck) * 4));
+  L.bstart = static_cast<uint32_t*>(cv.take(size_t(nbuck + 1) * 4));
+  L.istart = static_cast<uint32_t*>(cv.take(size_t(nbuck + 1) * 4));
+  L.entries = static_cast<int32_t*>(cv.take(size_t(max_entries) * 4));
+  L.items = static_cast<int4*>(cv.take(size_t(max_items) * 16));
+  L.opart = cv.take(size_t(max_entries) * R * d * 2);
+  L.lse = static_cast<float*>(cv.take(size_t(max_entries) * R * 4));
+  L.bytes = cv.off;
+  return L;
+}
+
+template <int D, int RP>
+msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                            const KvParams& kp, cudaStream_t st) {
+  using C = KvCfg<D, RP>;
+  static std::once_flag once;
+  static msa_status_t attr = MSA_OK;
+  std::call_once(once, [] { attr = set_smem(kvouter_kernel<D, RP>, C::kSmemBytes); });
+  if (attr != MSA_OK) return attr;
+  kvouter_kernel<D, RP><<<num_sms(), kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, kp);
+  MSA_CHECK_LAUNCH();
+  return MSA_OK;
+}
+
+template <int D>
+msa_status_t dispatch_kvouter(int R, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                              const CUtensorMap& to, const KvParams& kp, cudaStream_t st) {
+  if (R <= 8) return launch_kvouter<D, 8>(tq, tk, tv, to, kp, st);
+  return launch_kvouter<D, 16>(tq, tk, tv, to, kp, st);
+}
+
+msa_status_t set_csr_smem() {
+  static std::once_flag once;
+  static msa_status_t attr = MSA_OK;
+  std::call_once(once, [] {
+    attr = set_smem(csr_count_kernel, 227 * 1024);
+    if (attr == MSA_OK) attr = set_smem(csr_scatter_kernel, 227 * 1024);
+  });
+  return attr;
+}
+
+msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const int32_t* block_ids, int64_t n,
+                             int32_t hq, int32_t g, int32_t d, int32_t k, float scale, void* o, void* ws,
+                             int64_t query_chunk, cudaStream_t st) {
+  msa_status_t s;
+  if ((s = set_csr_smem()) != MSA_OK) return s;
+  const int R = hq / g;
+  const int RP = rows_per_query(R);
+  const int TQ = 128 / RP;
+  AttnLayout L = attn_layout(ws, n, hq, g, d, k, query_chunk);
+  const int64_t nb = (n + 127) / 128;
+  if (scale == 0.0f) scale = 1.0f / std::sqrt(float(d));
+  CUtensorMap tq, tk, tv, to;
+  if ((s = make_map_3d(&tq, q, d, hq, n, uint64_t(d) * 2, uint64_t(hq) * d * 2, 64, RP, 1,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  if ((s = make_map_3d(&tk, kk, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  if ((s = make_map_3d(&tv, v, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  const int64_t slot_rows = L.chunk_blocks * 128 * g * k;
+  if ((s = make_map_3d(&to, L.opart, d, R, slot_rows, uint64_t(d) * 2, uint64_t(R) * d * 2, 64, R, 1,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  for (int64_t qa0 = 0; qa0 < nb; qa0 += L.chunk_blocks) {
+    const int64_t qa1 = std::min(nb, qa0 + L.chunk_blocks);
+    CsrParams cp{};
+    cp.block_ids = block_ids;
+    cp.N = n;
+    cp.G = g;
+    cp.k = k;
+    cp.qa0 = int(qa0);
+    cp.qa1 = int(qa1);
+    cp.nt = int(qa1 - qa0);
+    cp.tq = TQ;
+    cp.item_tiles = kKvItemTiles;
+    cp.hist = L.hist;
+    cp.totals = L.totals;
+    cp.bucket_start = L.bstart;
+    cp.item_start = L.istart;
+    cp.entries = L.entries;
+    cp.items = L.items;
+    const int64_t nbuck = int64_t(g) * qa1;
+    const size_t bm_bytes = size_t(qa1) * 16;
+    if (bm_bytes > 227 * 1024) return fail(MSA_ERR_UNSUPPORTED, "sequence too long for the CSR build (%lld blocks)", (long long)qa1);
+    csr_count_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp);
+    MSA_CHECK_LAUNCH();
+    csr_scan_kernel<<<unsigned((nbuck + 7) / 8), 256, 0, st>>>(cp);
+    MSA_CHECK_LAUNCH();
+    csr_offsets_kernel<<<1, 1024, 0, st>>>(cp);
+    MSA_CHECK_LAUNCH();
+    csr_scatter_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp);
+    MSA_CHECK_LAUNCH();
+    csr_items_kernel<<<unsigned((nbuck + 255) / 256), 256, 0, st>>>(cp);
+    MSA_CHECK_LAUNCH();
+    KvParams kp{};
+    kp.entries = L.entries;
+    kp.items = L.items;
+    kp.n_items = L.istart + nbuck;
+    kp.G = g;
+    kp.R = R;
+    kp.k = k;
+    kp.nbk = int(qa1);
+    kp.row0 = qa0 * 128;
+    kp.scale_log2 = scale * 1.4426950408889634f;
+    kp.lse = L.lse;
+    if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, to, kp, st);
+    else s = dispatch_kvouter<64>(R, tq, tk, tv, to, kp, st);
+    if (s != MSA_OK) return s;
+    MergeParams mp{};
+    mp.opart = static_cast<const __nv_bfloat16*>(L.opart);
+    mp.lse = L.lse;
+    mp.block_ids = block_ids;
+    mp.o = static_cast<__nv_bfloat16*>(o);
+    mp.row0 = qa0 * 128;
+    mp.rows = std::min<int64_t>(n, qa1 * 128) - qa0 * 128;
+    mp.G = g;
+    mp.R = R;
+    mp.k = k;
+    const int hpw = 32 / (d / 8);
+    const int64_t warps = (mp.rows * g * R + hpw - 1) / hpw;
+    const unsigned blocks = unsigned((warps + 7) / 8);
+    if (d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
+    else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
+    MSA_CHECK_LAUNCH();
+  }
+  return MSA_OK;
+}
+
+// ------------------------------- decode -------------------------------
+struct DecodeLayout {
+  uint32_t* maxima = nullptr;
+  int32_t* block_ids = nullptr;
+  void* opart = nullptr;
+  float* lse = nullptr;
+  size_t bytes = 0;
+};
+
+DecodeLayout decode_layout(void* ws, const msa_params* p, bool need_ids) {
+  const int64_t B = p->n;
+  const int64_t nbmax = (p->lmax + 127) / 128;
+  const int R = p->hq / p->g;
+  Carver cv(ws);
+  DecodeLayout L;
+  L.maxima = static_cast<uint32_t*>(cv.take(size_t(B) * p->g * nbmax * 4));
+  if (need_ids) L.block_ids = static_cast<int32_t*>(cv.take(size_t(B) * p->g * p->k * 4));
+  L.opart = cv.take(size_t(B) * p->g * p->k * R * p->d * 2);
+  L.lse = static_cast<float*>(cv.take(size_t(B) * p->g * p->k * R * 4));
+  L.bytes = cv.off;
+  return L;
+}
+
+msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, const void* vc, const void* q_idx,
+                        const void* k_idx, int32_t* block_ids_out, void* o, void* ws, cudaStream_t st) {
+  DecodeLayout L = decode_layout(ws, p, block_ids_out == nullptr);
+  int32_t* ids = block_ids_out ? block_ids_out : L.block_ids;
+  const int B = int(p->n);
+  const int nbmax = int((p->lmax + 127) / 128);
+  const int R = p->hq / p->g;
+  const float scale = p->scale == 0.0f ? 1.0f / std::sqrt(float(p->d)) : p->scale;
+  DecodeScanParams sp{};
+  sp.q_idx = static_cast<const __nv_bfloat16*>(q_idx);
+  sp.k_idx = static_cast<const __nv_bfloat16*>(k_idx);
+  sp.seqlens = p->seqlens;
+  sp.maxima = L.maxima;
+  sp.B = B;
+  sp.G = p->g;
+  sp.nbmax = nbmax;
+  sp.Lmax = p->lmax;
+  const dim3 sgrid(nbmax, B);
+  switch (p->d_idx) {
+    case 32: decode_scan_kernel<32><<<sgrid, 256, 0, st>>>(sp); break;
+    case 64: decode_scan_kernel<64><<<sgrid, 256, 0, st>>>(sp); break;
+    case 128: decode_scan_kernel<128><<<sgrid, 256, 0, st>>>(sp); break;
+    default: return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d", p->d_idx);
+  }
+  MSA_CHECK_LAUNCH();
+  TopkDecodeParams tp{};
+  tp.maxima = L.maxima;
+  tp.block_ids = ids;
+  tp.seqlens = p->seqlens;
+  tp.B = B;
+  tp.G = p->g;
+  tp.k = p->k;
+  tp.nbmax = nbmax;
+  msa_status_t s;
+  if ((s = dispatch_topk_decode(p->k, tp, st)) != MSA_OK) return s;
+  MSA_CHECK_LAUNCH();
+  DecodeAttnParams ap{};
+  ap.q = static_cast<const __nv_bfloat16*>(q);
+  ap.kc = static_cast<const __nv_bfloat16*>(kc);
+  ap.vc = static_cast<const __nv_bfloat16*>(vc);
+  ap.seqlens = p->seqlens;
+  ap.block_ids = ids;
+  ap.opart = static_cast<__nv_bfloat16*>(L.opart);
+  ap.lse = L.lse;
+  ap.B = B;
+  ap.G = p->g;
+  ap.R = R;
+  ap.k = p->k;
+  ap.Lmax = p->lmax;
+  ap.scale_log2 = scale * 1.4426950408889634f;
+  const int smem = 2 * 128 * (p->d + 8) * 2 + R * p->d * 4 + R * 128 * 4 + R * 8;
+  const dim3 agrid(p->k, p->g, B);
+  if (p->d == 128) {
+    static std::once_flag once;
+    static msa_status_t attr = MSA_OK;
+    std::call_once(once, [] { attr = set_smem(decode_attn_kernel<128>, 200 * 1024); });
+    if (attr != MSA_OK) return attr;
+    decode_attn_kernel<128><<<agrid, 128, smem, st>>>(ap);
+  } else {
+    static std::once_flag once;
+    static msa_status_t attr = MSA_OK;
+    std::call_once(once, [] { attr = set_smem(decode_attn_kernel<64>, 200 * 1024); });
+    if (attr != MSA_OK) return attr;
+    decode_attn_kernel<64><<<agrid, 128, smem, st>>>(ap);
+  }
+  MSA_CHECK_LAUNCH();
+  MergeParams mp{};
+  mp.opart = static_cast<const __nv_bfloat16*>(L.opart);
+  mp.lse = L.lse;
+  mp.block_ids = ids;
+  mp.o = static_cast<__nv_bfloat16*>(o);
+  mp.row0 = 0;
+  mp.rows = B;
+  mp.G = p->g;
+  mp.R = R;
+  mp.k = p->k;
+  const int hpw = 32 / (p->d / 8);
+  const int64_t warps = (int64_t(B) * p->g * R + hpw - 1) / hpw;
+  const unsigned blocks = unsigned((warps + 7) / 8);
+  if (p->d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
+  else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
+  MSA_CHECK_LAUNCH();
+  return MSA_OK;
+}
+
+msa_status_t check_main_dims(int32_t hq, int32_t g, int32_t d) {
+  if (hq < 1 || hq % g != 0) return fail(MSA_ERR_INVALID_ARG, "hq=%d is not a positive multiple of g=%d", hq, g);
+  if (!supported_r(hq / g)) return fail(MSA_ERR_UNSUPPORTED, "hq/g=%d unsupported (1, 2, 4, 8, 16)", hq / g);
+  if (d != 64 && d != 128) return fail(MSA_ERR_UNSUPPORTED, "d=%d unsupported (64, 128)", d);
+  return MSA_OK;
+}
+
+msa_status_t check_d_idx(int32_t d_idx) {
+  if (d_idx != 32 && d_idx != 64 && d_idx != 128) return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d unsupported (32, 64, 128)", d_idx);
+  return MSA_OK;
+}
+
+size_t prefill_ids_bytes(int64_t n, int32_t g, int32_t k) { return align_up(size_t(n) * g * k * 4); }
+
+}  // namespace
+
+// =====================================================================================
+// C ABI
+// =====================================================================================
+extern "C" {
+
+const char* msa_status_string(msa_status_t s) {
+  switch (s) {
+    case MSA_OK: return "MSA_OK";
+    case MSA_ERR_INVALID_ARG: return "MSA_ERR_INVALID_ARG";
+    case MSA_ERR_UNSUPPORTED: return "MSA_ERR_UNSUPPORTED";
+    case MSA_ERR_WORKSPACE: return "MSA_ERR_WORKSPACE";
+    case MSA_ERR_CUDA: return "MSA_ERR_CUDA";
+    case MSA_ERR_TIMEOUT: return "MSA_ERR_TIMEOUT";
+    case MSA_ERR_DEVICE_BOUNDS: return "MSA_ERR_DEVICE_BOUNDS";
+  }
+  return "MSA_ERR_UNKNOWN";
+}
+
+const char* msa_last_error_detail(void) { return g_detail; }
+
+size_t msa_index_select_workspace(int64_t n, int32_t g, int32_t d_idx, int32_t bk, int32_t k) {
+  if (check_common(n, g, bk, k) != MSA_OK || check_d_idx(d_idx) != MSA_OK) return 0;
+  return index_layout(nullptr, n, g).bytes;
+}
+
+msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx, int32_t bk,
+                              int32_t k, int32_t* block_ids, void* workspace, size_t workspace_bytes, void* stream) {
+  g_detail[0] = 0;
+  msa_status_t s;
+  if ((s = check_common(n, g, bk, k)) != MSA_OK) return s;
+  if ((s = check_d_idx(d_idx)) != MSA_OK) return s;
+  if ((s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
+      (s = check_ptr(block_ids, "block_ids")) != MSA_OK || (s = check_ptr(workspace, "workspace")) != MSA_OK)
+    return s;
+  const size_t need = index_layout(nullptr, n, g).bytes;
+  if (workspace_bytes < need)
+    return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  return run_index_select(q_idx, k_idx, n, g, d_idx, k, block_ids, workspace, static_cast<cudaStream_t>(stream));
+}
+
+size_t msa_sparse_attn_workspace(int64_t n, int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t k) {
+  if (check_common(n, g, bk, k) != MSA_OK || check_main_dims(hq, g, d) != MSA_OK) return 0;
+  return attn_layout(nullptr, n, hq, g, d, k, 0).bytes;
+}
+
+msa_status_t msa_sparse_attn(const void* q, const void* k, const void* v, const int32_t* block_ids, int64_t n,
+                             int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t kk, float scale, void* o,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  g_detail[0] = 0;
+  msa_status_t s;
+  if ((s = check_common(n, g, bk, kk)) != MSA_OK) return s;
+  if ((s = check_main_dims(hq, g, d)) != MSA_OK) return s;
+  if (!(scale >= 0.0f) || std::isinf(scale)) return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if ((s = check_ptr(q, "q")) != MSA_OK || (s = check_ptr(k, "k")) != MSA_OK || (s = check_ptr(v, "v")) != MSA_OK ||
+      (s = check_ptr(block_ids, "block_ids")) != MSA_OK || (s = check_ptr(o, "o")) != MSA_OK ||
+      (s = check_ptr(workspace, "workspace")) != MSA_OK)
+    return s;
+  const size_t need = attn_layout(nullptr, n, hq, g, d, kk, 0).bytes;
+  if (workspace_bytes < need)
+    return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  return run_sparse_attn(q, k, v, block_ids, n, hq, g, d, kk, scale, o, workspace, 0,
+                         static_cast<cudaStream_t>(stream));
+}
+
+size_t msa_forward_workspace(const msa_params* p) {
+  if (!p) return 0;
+  if (p->mode == MSA_MODE_PREFILL) {
+    if (check_common(p->n, p->g, p->bk, p->k) != MSA_OK || check_main_dims(p->hq, p->g, p->d) != MSA_OK ||
+        check_d_idx(p->d_idx) != MSA_OK)
+      return 0;
+    if (p->query_chunk < 0 || p->query_chunk % 128 != 0) return 0;
+    const size_t a = attn_layout(nullptr, p->n, p->hq, p->g, p->d, p->k, p->query_chunk).bytes;
+    const size_t b = index_layout(nullptr, p->n, p->g).bytes;
+    return prefill_ids_bytes(p->n, p->g, p->k) + std::max(a, b);
+  }
+  if (p->mode == MSA_MODE_DECODE) {
+    if (check_common(p->n, p->g, p->bk, p->k) != MSA_OK || check_main_dims(p->hq, p->g, p->d) != MSA_OK ||
+        check_d_idx(p->d_idx) != MSA_OK || p->lmax < 1)
+      return 0;
+    return decode_layout(nullptr, p, true).bytes;
+  }
+  return 0;
+}
+
+msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, const void* v, const void* q_idx,
+                         const void* k_idx, int32_t* block_ids_out, void* o, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  g_detail[0] = 0;
+  if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
+  msa_status_t s;
+  if ((s = check_common(p->n, p->g, p->bk, p->k)) != MSA_OK) return s;
+  if ((s = check_main_dims(p->hq, p->g, p->d)) != MSA_OK) return s;
+  if ((s = check_d_idx(p->d_idx)) != MSA_OK) return s;
+  if (!(p->scale >= 0.0f) || std::isinf(p->scale)) return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if ((s = check_ptr(q, "q")) != MSA_OK || (s = check_ptr(k, "k")) != MSA_OK || (s = check_ptr(v, "v")) != MSA_OK ||
+      (s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
+      (s = check_ptr(o, "o")) != MSA_OK || (s = check_ptr(workspace, "workspace")) != MSA_OK)
+    return s;
+  if (block_ids_out && (s = check_ptr(block_ids_out, "block_ids_out")) != MSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p->mode == MSA_MODE_PREFILL) {
+    if (p->query_chunk < 0 || p->query_chunk % 128 != 0)
+      return fail(MSA_ERR_INVALID_ARG, "query_chunk=%lld must be a non-negative multiple of 128", (long long)p->query_chunk);
+    const size_t need = msa_forward_workspace(p);
+    if (workspace_bytes < need)
+      return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    int32_t* ids = block_ids_out ? block_ids_out : reinterpret_cast<int32_t*>(w);
+    void* rest = w + prefill_ids_bytes(p->n, p->g, p->k);
+    if ((s = run_index_select(q_idx, k_idx, p->n, p->g, p->d_idx, p->k, ids, rest, st)) != MSA_OK) return s;
+    return run_sparse_attn(q, k, v, ids, p->n, p->hq, p->g, p->d, p->k, p->scale, o, rest, p->query_chunk, st);
+  }
+  if (p->mode == MSA_MODE_DECODE) {
+    if (p->lmax < 1 || p->lmax > kMaxN) return fail(MSA_ERR_INVALID_ARG, "lmax=%lld out of range", (long long)p->lmax);
+    if ((s = check_ptr(p->seqlens, "seqlens")) != MSA_OK) return s;
+    const int cpt = p->g * p->d_idx / 32;
+    if (cpt > 32 || (cpt & (cpt - 1)) != 0)
+      return fail(MSA_ERR_UNSUPPORTED, "decode needs g*d_idx/32 a power of two <= 32 (got %d)", cpt);
+    if (p->n > 65535) return fail(MSA_ERR_UNSUPPORTED, "decode batch %lld > 65535", (long long)p->n);
+    const size_t need = msa_forward_workspace(p);
+    if (workspace_bytes < need)
+      return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+    return run_decode(p, q, k, v, q_idx, k_idx, block_ids_out, o, workspace, st);
+  }
+  return fail(MSA_ERR_INVALID_ARG, "mode=%d", p->mode);
+}
+
+msa_status_t msa_get_device_error(void* stream) {
+  g_detail[0] = 0;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  unsigned int v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, msa::g_msa_error, sizeof(v));
+  if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+  if (v != 0) {
+    e = cudaMemcpyToSymbol(msa::g_msa_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "clear error word: %s", cudaGetErrorString(e));
+    fail(static_cast<msa_status_t>(v & 0xFF), "device error %s in kernel %u", msa_status_string(static_cast<msa_status_t>(v & 0xFF)),
+         (v >> 8) & 0xFF);
+    return static_cast<msa_status_t>(v & 0xFF);
+  }
+  return MSA_OK;
+}
+
+}  // extern "C"

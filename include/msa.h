@@ -1,0 +1,133 @@
+/*
+ * msa.h — C ABI of the B200 (sm_100a) library for the hot path of MiniMax Sparse
+ * Attention (MSA).
+ *
+ * What the library computes (hyper.ai "MiniMax Sparse Attention", Method; zhichai.net
+ * article, section 2 "Index Branch" / "Main Branch"):
+ *   Index Branch, per GQA group g and query i:
+ *     s_g(i, j) = q_idx[i, g] . k_idx[j, g] for every causally visible token j <= i;
+ *     S_g(i, b) = max of s_g(i, j) over the tokens j <= i of block b (Block Max
+ *     Pooling, blocks of Bk = 128 tokens);
+ *     block_ids[i, g, :] = the local block b_l = floor(i / Bk) plus the k - 1 best other
+ *     visible blocks by S (higher first, lower block index first among equal scores);
+ *     when b_l + 1 <= k every visible block is taken. Rows list ids in ascending
+ *     order and are padded with -1.
+ *   Main Branch, per query head h of group g = h / (Hq / G):
+ *     o[i, h] = softmax(q[i, h] . k[j, g] * scale) . v[j, g] over the tokens j <= i of
+ *     the selected blocks (standard scaled dot-product attention, scale 1/sqrt(d)
+ *     unless given).
+ *   Decode applies the same definition to one new query per sequence, at position
+ *   seqlens[b] - 1 of that sequence's cache.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major and contiguous, bf16 passed as raw 16-bit storage
+ *     (const void*). Every pointer is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned. The library allocates and frees nothing; scratch memory comes from the
+ *     caller's workspace (size from the matching *_workspace function; 256-byte
+ *     aligned base).
+ *   - stream is a cudaStream_t (NULL = legacy default stream). All work is enqueued on
+ *     it; no call synchronises the host, except msa_get_device_error.
+ *   - Arguments are validated before anything is enqueued. A bad argument returns
+ *     MSA_ERR_INVALID_ARG, a valid but unimplemented shape MSA_ERR_UNSUPPORTED, a too
+ *     small workspace MSA_ERR_WORKSPACE, a failed CUDA launch MSA_ERR_CUDA; nothing is
+ *     launched in those cases. msa_last_error_detail() then describes the failure.
+ *   - Faults detected on the device (a pipeline wait that timed out, an index out of
+ *     range) are recorded in a per-device error word and reported by
+ *     msa_get_device_error(); the kernel that saw it returns early, so the output of
+ *     that call is undefined.
+ *   - Supported shapes: Bk = 128; d in {64, 128}; d_idx in {32, 64, 128};
+ *     R = Hq / G in {1, 2, 4, 8, 16}; 1 <= k <= 32; 1 <= N < 2^26.
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MSA_API __attribute__((visibility("default")))
+#else
+#define MSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum msa_status_t {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,
+  MSA_ERR_UNSUPPORTED = 2,
+  MSA_ERR_WORKSPACE = 3,
+  MSA_ERR_CUDA = 4,
+  MSA_ERR_TIMEOUT = 5,
+  MSA_ERR_DEVICE_BOUNDS = 6
+} msa_status_t;
+
+typedef enum msa_mode_t { MSA_MODE_PREFILL = 0, MSA_MODE_DECODE = 1 } msa_mode_t;
+
+/* Shapes of one msa_forward call.
+ *   prefill: n = N tokens of one sequence; q [N, hq, d]; k, v [N, g, d];
+ *            q_idx, k_idx [N, g, d_idx]; o [N, hq, d]; block_ids [N, g, k].
+ *   decode:  n = B sequences, one new query each; q [B, hq, d]; q_idx [B, g, d_idx];
+ *            caches k, v [B, lmax, g, d] and k_idx [B, lmax, g, d_idx], where the new
+ *            token's k / v / k_idx are already stored at position seqlens[b] - 1;
+ *            seqlens: device int32 [B], 1 <= seqlens[b] <= lmax; o [B, hq, d];
+ *            block_ids [B, g, k].
+ * query_chunk (prefill): queries per attention chunk, a multiple of 128; 0 picks the
+ * library default. Larger chunks use more workspace. */
+typedef struct msa_params {
+  int32_t mode;
+  int32_t hq, g, d, d_idx, bk, k;
+  float scale;               /* 0 => 1 / sqrt(d) */
+  int64_t n;
+  int64_t lmax;              /* decode only */
+  const int32_t* seqlens;    /* decode only, device pointer */
+  int64_t query_chunk;       /* prefill only */
+} msa_params;
+
+/* Index Branch (scores, Block Max Pooling, Top-k with the local block forced).
+ * q_idx, k_idx: [n, g, d_idx] bf16. block_ids (out): [n, g, k] int32.
+ * Returns MSA_OK or an error as described above. */
+MSA_API size_t msa_index_select_workspace(int64_t n, int32_t g, int32_t d_idx, int32_t bk, int32_t k);
+MSA_API msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx,
+                              int32_t bk, int32_t k, int32_t* block_ids, void* workspace,
+                              size_t workspace_bytes, void* stream);
+
+/* Main Branch given the selection, executed KV-outer (each K/V block is held on chip
+ * while the queries that chose it stream through; per-slot partial results are
+ * merged by a deterministic log-sum-exp pass, no atomics).
+ * q: [n, hq, d]; k, v: [n, g, d]; block_ids: [n, g, topk] as produced by
+ * msa_index_select (ascending, -1 padded, each id <= floor(i / bk)); o (out):
+ * [n, hq, d] bf16. scale 0 => 1 / sqrt(d). Ids that break the rules above are
+ * reported through msa_get_device_error as MSA_ERR_DEVICE_BOUNDS. */
+MSA_API size_t msa_sparse_attn_workspace(int64_t n, int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t topk);
+MSA_API msa_status_t msa_sparse_attn(const void* q, const void* k, const void* v, const int32_t* block_ids, int64_t n,
+                             int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t topk, float scale, void* o,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Both branches in one call: prefill (Index Branch then KV-outer Main Branch) or
+ * decode (query-stationary index scan, Top-k, sparse attention over the selected
+ * blocks, merge). block_ids_out may be NULL (the selection then lives in the
+ * workspace). */
+MSA_API size_t msa_forward_workspace(const msa_params* p);
+MSA_API msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, const void* v, const void* q_idx,
+                         const void* k_idx, int32_t* block_ids_out, void* o, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears this device's error word. Returns
+ * MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_DEVICE_BOUNDS (the first error recorded since the
+ * last call), or MSA_ERR_CUDA when the synchronisation itself failed. */
+MSA_API msa_status_t msa_get_device_error(void* stream);
+
+/* Static English name of a status code. */
+MSA_API const char* msa_status_string(msa_status_t status);
+
+/* Text of the last validation or launch failure seen by this host thread ("" if none). */
+MSA_API const char* msa_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

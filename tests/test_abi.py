@@ -1,0 +1,94 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared symbol, and
+rejects bad arguments synchronously (before any CUDA work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_tcgen05_b200 import build as msa_build
+from block_sparse_long_tcgen05_b200 import msa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "msa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    msa_build.build()
+    return msa.load_library()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"MSA_API\s+[\w\s\*]+?\b(msa_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_documented_entry_points():
+    names = declared_functions()
+    assert set(names) == set(msa.EXPORTS), names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_library_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {msa.LIB_PATH}").read()
+    exported = sorted(l.split()[-1] for l in out.splitlines() if " T " in l)
+    assert exported == sorted(declared_functions())
+
+
+def test_status_strings(lib):
+    for code, name in msa.STATUS.items():
+        assert lib.msa_status_string(code).decode() == name
+
+
+def test_validation_rejects_bad_arguments_without_cuda(lib):
+    P = 1 << 12  # an aligned fake address: never dereferenced, validation fails first
+    # NULL pointer
+    assert lib.msa_index_select(None, P, 256, 2, 32, 128, 4, P, P, 1 << 30, None) == 1
+    assert b"q_idx" in lib.msa_last_error_detail()
+    # misaligned pointer
+    assert lib.msa_index_select(P + 2, P, 256, 2, 32, 128, 4, P, P, 1 << 30, None) == 1
+    # unsupported block size, d_idx, k
+    assert lib.msa_index_select(P, P, 256, 2, 32, 64, 4, P, P, 1 << 30, None) == 2
+    assert lib.msa_index_select(P, P, 256, 2, 48, 128, 4, P, P, 1 << 30, None) == 2
+    assert lib.msa_index_select(P, P, 256, 2, 32, 128, 33, P, P, 1 << 30, None) == 2
+    # bad n
+    assert lib.msa_index_select(P, P, 0, 2, 32, 128, 4, P, P, 1 << 30, None) == 1
+    # workspace too small
+    need = lib.msa_index_select_workspace(4096, 2, 32, 128, 4)
+    assert need > 0
+    assert lib.msa_index_select(P, P, 4096, 2, 32, 128, 4, P, P, need - 1, None) == 3
+    # heads not a multiple of groups / unsupported ratio / unsupported d
+    assert lib.msa_sparse_attn(P, P, P, P, 256, 6, 4, 64, 128, 4, 0.0, P, P, 1 << 30, None) == 1
+    assert lib.msa_sparse_attn(P, P, P, P, 256, 12, 4, 64, 128, 4, 0.0, P, P, 1 << 30, None) == 2
+    assert lib.msa_sparse_attn(P, P, P, P, 256, 8, 2, 96, 128, 4, 0.0, P, P, 1 << 30, None) == 2
+    assert lib.msa_sparse_attn(P, P, P, P, 256, 8, 2, 64, 128, 4, -1.0, P, P, 1 << 30, None) == 1
+    assert lib.msa_sparse_attn(P, P, P, P, 256, 8, 2, 64, 128, 4, float("nan"), P, P, 1 << 30, None) == 1
+
+
+def test_forward_param_validation(lib):
+    P = 1 << 12
+    p = msa.prefill_params(1000, 8, 2, 64, 32, 4)
+    need = lib.msa_forward_workspace(ctypes.byref(p))
+    assert need > 0
+    p.query_chunk = 100   # not a multiple of 128
+    assert lib.msa_forward_workspace(ctypes.byref(p)) == 0
+    assert lib.msa_forward(ctypes.byref(p), P, P, P, P, P, None, P, P, 1 << 40, None) == 1
+    p.query_chunk = 0
+    p.mode = 7
+    assert lib.msa_forward(ctypes.byref(p), P, P, P, P, P, None, P, P, 1 << 40, None) == 1
+    d = msa.MsaParams(mode=1, hq=64, g=8, d=128, d_idx=128, bk=128, k=16, scale=0.0, n=4, lmax=1000,
+                      seqlens=None, query_chunk=0)
+    assert lib.msa_forward_workspace(ctypes.byref(d)) > 0
+    assert lib.msa_forward(ctypes.byref(d), P, P, P, P, P, None, P, P, 1 << 40, None) == 1   # seqlens NULL
+
+
+def test_workspace_sizes_grow_with_problem(lib):
+    a = lib.msa_sparse_attn_workspace(32768, 64, 8, 128, 128, 16)
+    b = lib.msa_sparse_attn_workspace(131072, 64, 8, 128, 128, 16)
+    assert 0 < a <= b
+    assert lib.msa_index_select_workspace(131072, 8, 128, 128, 16) >= 4 * 8 * 128 * (1024 * 1023 // 2)

@@ -1,0 +1,189 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Bars: block selections bit-exact; outputs within |o - o_ref| <= 2e-2 + 2e-2 |o_ref|
+elementwise (bf16 inputs, fp32 accumulation). Small cases check every row (several
+tiles and a ragged tail); the full-size workloads check seeded sampled rows that
+always include the edge rows {0, Bk-1, Bk, k*Bk-1, k*Bk, N-1}.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_tcgen05_b200 import msa, synth
+from oracle import msa_oracle as orc
+
+pytestmark = pytest.mark.gpu
+
+ATOL = 2e-2
+RTOL = 2e-2
+
+
+def assert_close(o_gpu, o_ref, what=""):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    err = np.abs(o_gpu - o_ref)
+    bound = ATOL + RTOL * np.abs(o_ref)
+    bad = err > bound
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; "
+                           f"max err {err.max():.3e}, worst excess {(err - bound).max():.3e}")
+
+
+def sample_rows(N, k, Bk=128, n=64, seed=0):
+    must = [0, Bk - 1, Bk, k * Bk - 1, k * Bk, N - 1]
+    rng = np.random.default_rng(seed)
+    extra = rng.choice(N, size=min(n, N), replace=False).tolist()
+    return sorted(set(x for x in must + extra if 0 <= x < N))
+
+
+def cfg_of(N, Hq, G, d, d_idx, k, hot=0.0, seed=77, idx_range=4):
+    return synth.PrefillConfig("t", N=N, Hq=Hq, G=G, d=d, d_idx=d_idx, k=k, idx_range=idx_range,
+                               hot_frac=hot, seed=seed)
+
+
+def check_prefill(cfg, rows=None, query_chunk=0, check_all_ids=True):
+    dev = torch.device("cuda")
+    inp = synth.prefill_inputs(cfg, device=dev)
+    ids_gpu = torch.empty(cfg.N, cfg.G, cfg.k, dtype=torch.int32, device=dev)
+    o = msa.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cfg.k, block_ids=ids_gpu,
+                    query_chunk=query_chunk)
+    msa.check_device_error()
+    if rows is None:
+        rows = list(range(cfg.N))
+    ids_ref, o_ref = orc.prefill_rows(inp, rows, cfg.Bk, cfg.k)
+    ids_g = ids_gpu.cpu().numpy()
+    np.testing.assert_array_equal(ids_g[rows], ids_ref)
+    if check_all_ids:
+        # structural rules on every row: count, ascending, local block present
+        i = np.arange(cfg.N)
+        bl = i // cfg.Bk
+        valid = ids_g >= 0
+        assert np.array_equal(valid.sum(-1), np.broadcast_to(np.minimum(cfg.k, bl + 1)[:, None], valid.shape[:2]))
+        last = np.take_along_axis(ids_g, (valid.sum(-1, keepdims=True) - 1), axis=-1)[..., 0]
+        assert np.array_equal(last, np.broadcast_to(bl[:, None], last.shape))
+    assert_close(o.float().cpu().numpy()[rows], o_ref, "prefill o")
+    return inp, ids_gpu, o
+
+
+# ---------------------------------------------------------------- Index Branch alone
+
+@pytest.mark.parametrize("N,G,d_idx,k", [(2048, 2, 32, 4), (2048 + 77, 3, 64, 8), (1500, 1, 128, 16),
+                                         (640, 2, 128, 1), (5000, 2, 128, 32)])
+def test_index_select_all_rows_bit_exact(cuda_ok, N, G, d_idx, k):
+    cfg = cfg_of(N, G, G, 64, d_idx, k, hot=0.05, idx_range=3)
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    ids = msa.msa_index_select(inp["q_idx"], inp["k_idx"], k)
+    msa.check_device_error()
+    ref, _ = orc.index_select_rows(inp["q_idx"].cpu(), inp["k_idx"].cpu(), range(N), 128, k)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref)
+
+
+def test_index_select_all_equal_scores_tie_rule(cuda_ok):
+    """Every block score equal: the lowest block indices win (plus the local block)."""
+    N, G, k = 3000, 2, 5
+    q_idx = torch.ones(N, G, 32, dtype=torch.bfloat16, device="cuda")
+    k_idx = torch.ones(N, G, 32, dtype=torch.bfloat16, device="cuda")
+    ids = msa.msa_index_select(q_idx, k_idx, k).cpu().numpy()
+    for i in (0, 127, 128, 600, 2999):
+        bl = i // 128
+        want = list(range(bl + 1))[:k] if bl + 1 <= k else [0, 1, 2, 3, bl]
+        want = want + [-1] * (k - len(want))
+        assert list(ids[i, 0]) == want and list(ids[i, 1]) == want
+
+
+def test_index_select_negative_zero_ties(cuda_ok):
+    """Scores of exactly zero from opposite-signed terms tie with plain zeros."""
+    N, G, k = 1024, 1, 3
+    q_idx = torch.zeros(N, G, 32, dtype=torch.bfloat16, device="cuda")
+    q_idx[:, :, 0] = 1
+    q_idx[:, :, 1] = 1
+    k_idx = torch.zeros(N, G, 32, dtype=torch.bfloat16, device="cuda")
+    k_idx[256:384, :, 0] = -1      # block 2: scores -1 + 1 = 0 (exact)
+    k_idx[256:384, :, 1] = 1
+    ids = msa.msa_index_select(q_idx, k_idx, k).cpu().numpy()
+    ref, _ = orc.index_select_rows(q_idx.cpu(), k_idx.cpu(), range(N), 128, k)
+    np.testing.assert_array_equal(ids, ref)
+
+
+# ---------------------------------------------------------------- Main Branch alone
+
+@pytest.mark.parametrize("N,Hq,G,d", [(2048, 8, 2, 64), (1000, 16, 2, 128), (777, 4, 4, 64),
+                                      (900, 32, 2, 128), (640, 4, 2, 128)])
+def test_sparse_attn_all_rows(cuda_ok, N, Hq, G, d):
+    cfg = cfg_of(N, Hq, G, d, 32, 4, seed=5)
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    ref_ids, _ = orc.index_select_rows(inp["q_idx"].cpu(), inp["k_idx"].cpu(), range(N), 128, 4)
+    ids = torch.from_numpy(ref_ids).cuda()
+    o = msa.msa_sparse_attn(inp["q"], inp["k"], inp["v"], ids)
+    msa.check_device_error()
+    o_ref = orc.attend_rows(inp["q"].cpu(), inp["k"].cpu(), inp["v"].cpu(), ref_ids, range(N), 128)
+    assert_close(o.float().cpu().numpy(), o_ref, "sparse_attn")
+
+
+def test_sparse_attn_rejects_bad_ids_on_device(cuda_ok):
+    """Ids above the query's own block are reported as MSA_ERR_DEVICE_BOUNDS (no fault)."""
+    cfg = cfg_of(512, 8, 2, 64, 32, 4)
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    ids = torch.full((512, 2, 4), -1, dtype=torch.int32, device="cuda")
+    ids[:, :, 0] = torch.div(torch.arange(512, device="cuda"), 128, rounding_mode="floor")[:, None].int()
+    ids[5, 1, 0] = 3                     # row 5 lives in block 0
+    msa.msa_sparse_attn(inp["q"], inp["k"], inp["v"], ids)
+    assert msa.msa_get_device_error() == 6
+    assert msa.msa_get_device_error() == 0   # cleared
+
+
+# ---------------------------------------------------------------- both branches
+
+def test_forward_tiny_config_all_rows(cuda_ok):
+    """The 2K tiny configuration (Hq=8, G=2, d=64, d_idx=32, k=4): every row."""
+    check_prefill(synth.TINY)
+
+
+def test_forward_dense_reduction(cuda_ok):
+    """k * Bk covering the context: MSA equals dense causal GQA (oracle, fp64)."""
+    cfg = cfg_of(1024 + 50, 8, 2, 64, 32, 9)
+    check_prefill(cfg)
+
+
+@pytest.mark.parametrize("query_chunk", [128, 256, 384])
+def test_forward_query_chunks(cuda_ok, query_chunk):
+    cfg = cfg_of(1300, 16, 2, 128, 64, 4, hot=0.1)
+    check_prefill(cfg, query_chunk=query_chunk)
+
+
+def test_forward_32k_sampled(cuda_ok):
+    check_prefill(synth.P32K, rows=sample_rows(32768, 16, n=96, seed=1))
+
+
+@pytest.mark.slow
+def test_forward_128k_sampled(cuda_ok):
+    """The headline 128K configuration, in the launch configuration the bench times."""
+    check_prefill(synth.P128K, rows=sample_rows(131072, 16, n=48, seed=2), check_all_ids=True)
+
+
+# ---------------------------------------------------------------- decode
+
+def check_decode(cfg, lengths, seqs=None, Lmax=None):
+    inp = synth.decode_inputs(cfg, device="cuda", lengths=lengths, Lmax=Lmax)
+    ids = torch.empty(len(lengths), cfg.G, cfg.k, dtype=torch.int32, device="cuda")
+    o = msa.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["q_idx"], inp["k_idx_cache"], inp["seqlens"],
+                   cfg.k, block_ids=ids)
+    msa.check_device_error()
+    seqs = list(range(len(lengths))) if seqs is None else seqs
+    ids_ref, o_ref = orc.decode_rows(inp, seqs, cfg.Bk, cfg.k)
+    np.testing.assert_array_equal(ids.cpu().numpy()[seqs], ids_ref)
+    assert_close(o.float().cpu().numpy()[seqs], o_ref, "decode o")
+
+
+def test_decode_varied_lengths(cuda_ok):
+    cfg = synth.DecodeConfig("t", B=9, L=0, Hq=64, G=8, d=128, d_idx=128, k=16, hot_frac=0.05, seed=9)
+    check_decode(cfg, [1, 2, 127, 128, 129, 2048, 2049, 5000, 9000], Lmax=9001)
+
+
+def test_decode_small_dims(cuda_ok):
+    cfg = synth.DecodeConfig("t", B=5, L=0, Hq=8, G=2, d=64, d_idx=32, k=4, hot_frac=0.0, seed=10, idx_range=3)
+    check_decode(cfg, [300, 700, 128, 1, 4096])
+
+
+@pytest.mark.slow
+def test_decode_full_size_sampled(cuda_ok):
+    """Batch 64 x 131073 tokens (the decode configuration); the oracle checks 6 sequences."""
+    check_decode(synth.DEC128K, [131073] * 64, seqs=[0, 1, 17, 31, 48, 63])
