@@ -1,0 +1,369 @@
+"""Benchmark of the MSA hot path on B200: prefill tokens/s and TFLOP/s at 128K, decode tokens/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one msa_forward prefill over the 131072-token sequence (Index Branch: scores +
+block max + Top-k; Main Branch: CSR build + KV-outer attention + LSE merge), inputs
+resident in HBM. Under torchrun every rank runs its own independent sequence (weak
+scaling, no data-path collective); the time is the max over ranks. Rank 0 prints one
+JSON line. `--impl reference` times the fp64 CPU oracle on a bounded sample of query
+rows of the same workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_tcgen05_b200 import accounting, synth  # noqa: E402
+
+METRIC = "prefill tokens/s & TFLOP/s (frac of bf16 peak) at 128K; decode tokens/s"
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def source_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "block_sparse_long_tcgen05_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        h.update(f.encode())
+        h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK), "fallback"
+
+
+# ------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) of one GPU during a timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------ dist
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------ CPU oracle
+def oracle_sample(inp: dict, cfg, rows: int, seed: int):
+    """Time the oracle (as it stands) on `rows` seeded query rows; returns (rows/s, seconds)."""
+    from oracle import msa_oracle as orc  # test / baseline infrastructure only
+    rng = np.random.default_rng(seed)
+    sel = sorted(rng.choice(cfg.N, size=rows, replace=False).tolist())
+    host = {n: t.detach().cpu() for n, t in inp.items()}
+    t0 = time.perf_counter()
+    orc.prefill_rows(host, sel, cfg.Bk, cfg.k)
+    dt = time.perf_counter() - t0
+    return rows / dt, dt
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def workload_config(cfg, extra=None) -> dict:
+    c = {"workload": cfg.name, "N": cfg.N, "Hq": cfg.Hq, "G": cfg.G, "d": cfg.d, "d_idx": cfg.d_idx,
+         "Bk": cfg.Bk, "k": cfg.k, "hot_frac": cfg.hot_frac, "seed": cfg.seed,
+         "l2": "inputs larger than L2 (q alone is 2.1 GB), no flush needed",
+         "parallelism": "one independent sequence per GPU, no collective"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    cfg = synth.CONFIGS[args.workload]
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = synth.prefill_inputs(cfg, device=dev)
+    rows = args.ref_rows
+    for w in range(args.warmup):
+        oracle_sample(inp, cfg, rows, seed=100 + w)
+    times = []
+    for s in range(args.steps):
+        _, dt = oracle_sample(inp, cfg, rows, seed=200 + s)
+        times.append(dt)
+    tot = sum(times)
+    value = rows * args.steps / tot
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{rows} seeded query rows of the {cfg.name} workload per step "
+                                       f"(both branches, fp64)"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ ours
+def timed(fn, steps: int, stream) -> float:
+    """ms per call of fn over `steps` calls, CUDA events on the launching stream."""
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def run_ours(args, world, rank, local):
+    from block_sparse_long_tcgen05_b200 import msa
+    msa.load_library()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks, peak_src = load_peaks()
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.prefill_inputs(cfg, device=dev, seed=cfg.seed + 7 * rank)
+    N = cfg.N
+    p = msa.prefill_params(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k)
+    ws = torch.empty(msa.msa_forward_workspace(p), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(inp["q"])
+    ids = torch.empty(N, cfg.G, cfg.k, dtype=torch.int32, device=dev)
+
+    def step():
+        msa.msa_forward(p, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], o=o, block_ids=ids,
+                        workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    msa.check_device_error(dev)
+    barrier(world)
+    clocks = ClockSampler(local) if rank == 0 else None
+    msa.msa_profile_start()
+    ms = timed(step, args.steps, stream)
+    stats = msa.msa_profile_stop()
+    clk = clocks.stop() if clocks else None
+    msa.check_device_error(dev)
+    ms = max_over_ranks(ms, world)
+    barrier(world)
+
+    idx_f, main_f = accounting.prefill_useful_flops(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.Bk, cfg.k)
+    useful_tflops = (idx_f + main_f) / (ms * 1e-3) / 1e12
+    value = world * N / (ms * 1e-3)
+
+    # per-kernel breakdown (this rank, same timed region)
+    stages = {}
+    total_stage_ms = sum(v[1] for v in stats.values())
+    for name, (launches, tot) in sorted(stats.items(), key=lambda kv: -kv[1][1]):
+        stages[name] = {"launches_per_step": launches / args.steps, "ms_per_step": tot / args.steps,
+                        "share": tot / total_stage_ms if total_stage_ms else None}
+    gpu_launches = sum(v[0] for v in stats.values())
+    nb = (N + 127) // 128
+    dom = max(stats.items(), key=lambda kv: kv[1][1])[0]
+    dom_launches, dom_ms = stats[dom]
+    per_launch_ms = dom_ms / dom_launches
+    traffic = args.traffic.get(dom) if args.traffic else None
+    if dom == "index_blockmax":
+        work = accounting.index_kernel_flops(0, nb, cfg.G, cfg.d_idx) / (dom_launches / args.steps)
+        ach = work / (per_launch_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
+                "work_per_launch": work}
+    elif dom == "kvouter":
+        work = accounting.kvouter_flops(N, cfg.Hq, cfg.d, cfg.Bk, cfg.k) / (dom_launches / args.steps)
+        ach = work / (per_launch_ms * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
+                "peak_source": f"{peak_src} bf16 sustained", "work_per_launch": work}
+    else:
+        byts = accounting.main_branch_bytes(N, cfg.Hq, cfg.G, cfg.d, cfg.Bk, cfg.k).get(dom, float("nan"))
+        work = byts / (dom_launches / args.steps)
+        ach = work / (per_launch_ms * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": f"{peak_src} HBM copy",
+                "work_per_launch": work}
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
+            "config": workload_config(cfg),
+            "prefill": {"tokens_per_s": value, "useful_tflops": useful_tflops * world,
+                        "useful_tflops_per_gpu": useful_tflops,
+                        "frac_spec_bf16_2250": useful_tflops / SPEC_BF16_TFLOPS,
+                        "frac_measured_bf16_burst": useful_tflops / peaks["bf16_tflops"],
+                        "frac_measured_bf16_sustained": useful_tflops / peaks["bf16_tflops_sustained"],
+                        "useful_tflop_per_step": (idx_f + main_f) / 1e12},
+            "stages": stages, "roofline": roof, "gpu_launches": gpu_launches, "clocks": clk}
+
+    # ------------------------------------------------ decode (query-stationary), same ranks
+    if not args.no_decode:
+        dcfg = synth.DEC128K
+        dinp = synth.decode_inputs(dcfg, device=dev, seed=dcfg.seed + 7 * rank)
+        dp = msa.decode_params(dcfg.B, dinp["k_cache"].shape[1], dinp["seqlens"], dcfg.Hq, dcfg.G, dcfg.d,
+                               dcfg.d_idx, dcfg.k)
+        dws = torch.empty(msa.msa_forward_workspace(dp), dtype=torch.uint8, device=dev)
+        do = torch.empty_like(dinp["q"])
+
+        def dstep():
+            msa.msa_forward(dp, dinp["q"], dinp["k_cache"], dinp["v_cache"], dinp["q_idx"],
+                            dinp["k_idx_cache"], o=do, workspace=dws)
+
+        for _ in range(max(3, args.warmup)):
+            dstep()
+        msa.check_device_error(dev)
+        barrier(world)
+        msa.msa_profile_start()
+        dms = timed(dstep, args.steps, stream)
+        dstats = msa.msa_profile_stop()
+        dms = max_over_ranks(dms, world)
+        scan_ms = dstats.get("decode_scan", (1, float("nan")))[1] / args.steps
+        scan_bytes = accounting.decode_scan_bytes([dcfg.L] * dcfg.B, dcfg.G, dcfg.d_idx)
+        d_idx_f, d_main_f = accounting.decode_useful_flops([dcfg.L] * dcfg.B, dcfg.Hq, dcfg.G, dcfg.d,
+                                                           dcfg.d_idx, dcfg.Bk, dcfg.k)
+        line["decode"] = {"workload": dcfg.name, "tokens_per_s": world * dcfg.B / (dms * 1e-3),
+                          "ms_per_step": dms, "useful_tflops_per_gpu": (d_idx_f + d_main_f) / (dms * 1e-3) / 1e12,
+                          "scan_hbm_gbs": scan_bytes / (scan_ms * 1e-3) / 1e9,
+                          "scan_frac_hbm": scan_bytes / (scan_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                          "stages": {k: {"ms_per_step": v[1] / args.steps} for k, v in dstats.items()}}
+        del dinp, dws, do
+        torch.cuda.empty_cache()
+
+    # ------------------------------------------------ end to end from pinned host memory
+    if not args.no_e2e:
+        host = {n: t.cpu().pin_memory() for n, t in inp.items()}
+        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = o_h.numel() * o_h.element_size()
+
+        def estep():
+            for n, t in host.items():
+                inp[n].copy_(t, non_blocking=True)
+            step()
+            o_h.copy_(o, non_blocking=True)
+
+        estep()
+        barrier(world)
+        esteps = max(2, min(args.steps, 10))
+        ems = max_over_ranks(timed(estep, esteps, stream), world)
+        line["e2e"] = {"value": world * N / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": esteps}
+
+    # ------------------------------------------------ CPU oracle baseline (rank 0, N = 1)
+    if world == 1 and not args.no_cpu_baseline:
+        rate, dt = oracle_sample(inp, cfg, args.ref_rows * 2, seed=7)
+        line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"{args.ref_rows * 2} seeded query rows of {cfg.name} "
+                                          f"(both branches, fp64), {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill-128k", choices=[c for c in synth.CONFIGS if "prefill" in c])
+    ap.add_argument("--ref-rows", type=int, default=8)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"),
+                    help="per-kernel DRAM bytes per launch from an ncu capture (null when absent)")
+    args = ap.parse_args()
+    args.traffic = {}
+    if args.traffic_json and os.path.exists(args.traffic_json):
+        tj = json.load(open(args.traffic_json))
+        # counters only describe the kernels they were taken on: drop them once the source changed
+        if tj.get("source_sha256") == source_sha256():
+            args.traffic = tj.get(args.workload, {})
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

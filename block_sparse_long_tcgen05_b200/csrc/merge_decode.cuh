@@ -22,7 +22,7 @@ struct MergeParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams P) {
+__global__ void __launch_bounds__(256, 2) merge_kernel(const __grid_constant__ MergeParams P) {
   constexpr int LPH = D / 8;          // lanes per head row (16 bytes each)
   constexpr int HPW = 32 / LPH;       // head rows per warp
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -35,26 +35,61 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
   const int64_t il = hh / (static_cast<int64_t>(P.R) * P.G);
   const int64_t i = P.row0 + il;
   const int32_t* ids = P.block_ids + (i * P.G + g) * P.k;
-  int nv = 0;
-  while (nv < P.k && ids[nv] >= 0) ++nv;
   const int64_t slot0 = (il * P.G + g) * P.k;
-  float L = -INFINITY;
-  for (int s = 0; s < nv; ++s) L = fmaxf(L, P.lse[(slot0 + s) * P.R + r]);
+  const uint4* prow = reinterpret_cast<const uint4*>(P.opart + (slot0 * P.R + r) * D) + c;
+  const int64_t pstride = static_cast<int64_t>(P.R) * D / 8;   // uint4 per slot
+  // The LPH lanes of this head row own slots c, c + LPH, ... for ids and lse. Every load of
+  // the row (ids, lse and the partials of the first 16 slots) is issued before any is
+  // used, so a row costs one memory round trip; slots past the valid ones are loaded but
+  // never used (they hold no partial).
+  const unsigned gmask = (LPH == 32) ? 0xffffffffu : (((1u << LPH) - 1u) << (lane & ~(LPH - 1)));
+  const int lane0 = lane & ~(LPH - 1);
+  int idv[4];
+  float own[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int s = c + LPH * j;
+    idv[j] = (s < P.k) ? __ldg(ids + s) : -1;
+    own[j] = (s < P.k) ? __ldg(P.lse + (slot0 + s) * P.R + r) : -INFINITY;
+  }
+  uint4 raw[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) raw[u] = (u < P.k) ? __ldg(prow + u * pstride) : make_uint4(0, 0, 0, 0);
+  int nv = 0;   // valid ids come first (ascending, -1 padded)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) nv += __popc(__ballot_sync(gmask, idv[j] >= 0) & gmask);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) own[j] = (c + LPH * j < nv) ? own[j] : -INFINITY;
+  float L = fmaxf(fmaxf(own[0], own[1]), fmaxf(own[2], own[3]));
+#pragma unroll
+  for (int o = 1; o < LPH; o <<= 1) L = fmaxf(L, __shfl_xor_sync(gmask, L, o));
+#pragma unroll
+  for (int j = 0; j < 4; ++j) own[j] = (c + LPH * j < nv) ? __expf(own[j] - L) : 0.0f;
   float acc[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
   float W = 0.0f;
-  for (int s = 0; s < nv; ++s) {
-    const float w = __expf(P.lse[(slot0 + s) * P.R + r] - L);
-    W += w;
-    const uint4 raw = __ldg(reinterpret_cast<const uint4*>(P.opart + ((slot0 + s) * P.R + r) * D) + c);
-    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+  auto accumulate = [&](const uint4& rw, int s) {   // ascending slot order
+    const int j = s / LPH;
+    const float mine = (j == 0) ? own[0] : (j == 1) ? own[1] : (j == 2) ? own[2] : own[3];
+    const float wu = __shfl_sync(gmask, mine, lane0 + (s % LPH));
+    if (s < nv) {
+      W += wu;
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&rw);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float2 f = __bfloat1622float2(h2[u]);
-      acc[2 * u] = fmaf(w, f.x, acc[2 * u]);
-      acc[2 * u + 1] = fmaf(w, f.y, acc[2 * u + 1]);
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(h2[t]);
+        acc[2 * t] = fmaf(wu, f.x, acc[2 * t]);
+        acc[2 * t + 1] = fmaf(wu, f.y, acc[2 * t + 1]);
+      }
     }
+  };
+#pragma unroll
+  for (int u = 0; u < 16; ++u) accumulate(raw[u], u);
+#pragma unroll 1
+  for (int s = 16; s < P.k; ++s) {   // k > 16: the remaining slots one by one (uniform trip count)
+    const uint4 rw = (s < nv) ? __ldg(prow + s * pstride) : make_uint4(0, 0, 0, 0);
+    accumulate(rw, s);
   }
   const float inv = (W > 0.0f) ? 1.0f / W : 0.0f;
   uint4 out;

@@ -141,6 +141,22 @@ msa_status_t make_map_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64
   return MSA_OK;
 }
 
+// 4-D bf16 tensor map: dims {d0..d3} (d0 innermost), byte strides of dims 1..3 (any order).
+msa_status_t make_map_4d(CUtensorMap* map, const void* base, const uint64_t (&dims)[4], const uint64_t (&strides)[3],
+                         const uint32_t (&box)[4], CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t d[4] = {dims[0], dims[1], dims[2], dims[3]};
+  const cuuint64_t s[3] = {strides[0], strides[1], strides[2]};
+  const cuuint32_t b[4] = {box[0], box[1], box[2], box[3]};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), d, s, b, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MSA_ERR_CUDA, "cuTensorMapEncodeTiled (4-D) failed (%d)", int(r));
+  return MSA_OK;
+}
+
 int num_sms() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
@@ -153,6 +169,58 @@ msa_status_t set_smem(K kernel, int bytes) {
   if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "cudaFuncSetAttribute(smem=%d): %s", bytes, cudaGetErrorString(e));
   return MSA_OK;
 }
+
+
+// ------------------------------- per-kernel timing -------------------------------
+enum ProfKind {
+  kPIndex, kPTopkPrefill, kPCsrCount, kPCsrScan, kPCsrOffsets, kPCsrScatter, kPCsrItems, kPKvOuter, kPMerge,
+  kPDecodeScan, kPTopkDecode, kPDecodeAttn, kPNumKinds
+};
+const char* const kProfNames[kPNumKinds] = {"index_blockmax", "topk_prefill", "csr_count", "csr_scan",
+                                            "csr_offsets", "csr_scatter", "csr_items", "kvouter", "merge",
+                                            "decode_scan", "topk_decode", "decode_attn"};
+struct ProfRec {
+  int kind;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t prof_event() {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Records a CUDA event before and after the launches of its scope when profiling is on.
+struct ProfScope {
+  ProfRec r{};
+  cudaStream_t st;
+  bool on;
+  ProfScope(int kind, cudaStream_t s) : st(s), on(g_prof_on) {
+    if (on) {
+      r.kind = kind;
+      r.a = prof_event();
+      r.b = prof_event();
+      cudaEventRecord(r.a, st);
+    }
+  }
+  ~ProfScope() {
+    if (on) {
+      cudaEventRecord(r.b, st);
+      std::lock_guard<std::mutex> lk(g_prof_mu);
+      g_prof.push_back(r);
+    }
+  }
+};
 
 // ------------------------------- index branch -------------------------------
 struct IndexLayout {
@@ -262,6 +330,7 @@ msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32
     const int64_t total = int64_t(acc) * g;
     if (total > 0) {
       const int grid = int(std::min<int64_t>(sms, total));
+      ProfScope ps(kPIndex, st);
       index_blockmax_kernel<DI><<<grid, kIdxThreads, C::kSmemBytes, st>>>(tq, tk, P, T);
       MSA_CHECK_LAUNCH();
     }
@@ -273,7 +342,10 @@ msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32
     tp.k = k;
     tp.qb0 = qb0;
     tp.region_per_group = P.region_per_group;
-    if ((s = dispatch_topk_prefill(k, tp, dim3(qb1 - qb0, g), st)) != MSA_OK) return s;
+    {
+      ProfScope ps(kPTopkPrefill, st);
+      if ((s = dispatch_topk_prefill(k, tp, dim3(qb1 - qb0, g), st)) != MSA_OK) return s;
+    }
     MSA_CHECK_LAUNCH();
   }
   return MSA_OK;
@@ -336,6 +408,7 @@ msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const 
   static msa_status_t attr = MSA_OK;
   std::call_once(once, [] { attr = set_smem(kvouter_kernel<D, RP>, C::kSmemBytes); });
   if (attr != MSA_OK) return attr;
+  ProfScope ps(kPKvOuter, st);
   kvouter_kernel<D, RP><<<num_sms(), kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, kp);
   MSA_CHECK_LAUNCH();
   return MSA_OK;
@@ -370,7 +443,10 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
   const int64_t nb = (n + 127) / 128;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(float(d));
   CUtensorMap tq, tk, tv, to;
-  if ((s = make_map_3d(&tq, q, d, hq, n, uint64_t(d) * 2, uint64_t(hq) * d * 2, 64, RP, 1,
+  const uint64_t panels = uint64_t(d) / 64;
+  // q as (64 elems, hq heads, panels, n): one box = 8 heads x all panels of one query
+  if ((s = make_map_4d(&tq, q, {64, uint64_t(hq), panels, uint64_t(n)},
+                       {uint64_t(d) * 2, 128, uint64_t(hq) * d * 2}, {64, 8, uint32_t(panels), 1},
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
   if ((s = make_map_3d(&tk, kk, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
@@ -380,7 +456,11 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
   const int64_t slot_rows = L.chunk_blocks * 128 * g * k;
-  if ((s = make_map_3d(&to, L.opart, d, R, slot_rows, uint64_t(d) * 2, uint64_t(R) * d * 2, 64, R, 1,
+  // partials [rows][R][d] as (64 elems, R heads, panels, rows); R >= 8: one box per 8 heads
+  // covering all panels, R < 8: one box per panel
+  if ((s = make_map_4d(&to, L.opart, {64, uint64_t(R), panels, uint64_t(slot_rows)},
+                       {uint64_t(d) * 2, 128, uint64_t(R) * d * 2},
+                       {64, uint32_t(std::min(R, 8)), R >= 8 ? uint32_t(panels) : 1u, 1},
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
   for (int64_t qa0 = 0; qa0 < nb; qa0 += L.chunk_blocks) {
@@ -404,15 +484,15 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     const int64_t nbuck = int64_t(g) * qa1;
     const size_t bm_bytes = size_t(qa1) * 16;
     if (bm_bytes > 227 * 1024) return fail(MSA_ERR_UNSUPPORTED, "sequence too long for the CSR build (%lld blocks)", (long long)qa1);
-    csr_count_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp);
+    { ProfScope ps(kPCsrCount, st); csr_count_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp); }
     MSA_CHECK_LAUNCH();
-    csr_scan_kernel<<<unsigned((nbuck + 7) / 8), 256, 0, st>>>(cp);
+    { ProfScope ps(kPCsrScan, st); csr_scan_kernel<<<unsigned((nbuck + 7) / 8), 256, 0, st>>>(cp); }
     MSA_CHECK_LAUNCH();
-    csr_offsets_kernel<<<1, 1024, 0, st>>>(cp);
+    { ProfScope ps(kPCsrOffsets, st); csr_offsets_kernel<<<1, 1024, 0, st>>>(cp); }
     MSA_CHECK_LAUNCH();
-    csr_scatter_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp);
+    { ProfScope ps(kPCsrScatter, st); csr_scatter_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp); }
     MSA_CHECK_LAUNCH();
-    csr_items_kernel<<<unsigned((nbuck + 255) / 256), 256, 0, st>>>(cp);
+    { ProfScope ps(kPCsrItems, st); csr_items_kernel<<<unsigned((nbuck + 255) / 256), 256, 0, st>>>(cp); }
     MSA_CHECK_LAUNCH();
     KvParams kp{};
     kp.entries = L.entries;
@@ -441,8 +521,11 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     const int hpw = 32 / (d / 8);
     const int64_t warps = (mp.rows * g * R + hpw - 1) / hpw;
     const unsigned blocks = unsigned((warps + 7) / 8);
-    if (d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
-    else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
+    {
+      ProfScope ps(kPMerge, st);
+      if (d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
+      else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
+    }
     MSA_CHECK_LAUNCH();
   }
   return MSA_OK;
@@ -489,11 +572,14 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   sp.nbmax = nbmax;
   sp.Lmax = p->lmax;
   const dim3 sgrid(nbmax, B);
-  switch (p->d_idx) {
-    case 32: decode_scan_kernel<32><<<sgrid, 256, 0, st>>>(sp); break;
-    case 64: decode_scan_kernel<64><<<sgrid, 256, 0, st>>>(sp); break;
-    case 128: decode_scan_kernel<128><<<sgrid, 256, 0, st>>>(sp); break;
-    default: return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d", p->d_idx);
+  {
+    ProfScope ps(kPDecodeScan, st);
+    switch (p->d_idx) {
+      case 32: decode_scan_kernel<32><<<sgrid, 256, 0, st>>>(sp); break;
+      case 64: decode_scan_kernel<64><<<sgrid, 256, 0, st>>>(sp); break;
+      case 128: decode_scan_kernel<128><<<sgrid, 256, 0, st>>>(sp); break;
+      default: return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d", p->d_idx);
+    }
   }
   MSA_CHECK_LAUNCH();
   TopkDecodeParams tp{};
@@ -505,7 +591,10 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   tp.k = p->k;
   tp.nbmax = nbmax;
   msa_status_t s;
-  if ((s = dispatch_topk_decode(p->k, tp, st)) != MSA_OK) return s;
+  {
+    ProfScope ps(kPTopkDecode, st);
+    if ((s = dispatch_topk_decode(p->k, tp, st)) != MSA_OK) return s;
+  }
   MSA_CHECK_LAUNCH();
   DecodeAttnParams ap{};
   ap.q = static_cast<const __nv_bfloat16*>(q);
@@ -528,12 +617,14 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
     static msa_status_t attr = MSA_OK;
     std::call_once(once, [] { attr = set_smem(decode_attn_kernel<128>, 200 * 1024); });
     if (attr != MSA_OK) return attr;
+    ProfScope ps(kPDecodeAttn, st);
     decode_attn_kernel<128><<<agrid, 128, smem, st>>>(ap);
   } else {
     static std::once_flag once;
     static msa_status_t attr = MSA_OK;
     std::call_once(once, [] { attr = set_smem(decode_attn_kernel<64>, 200 * 1024); });
     if (attr != MSA_OK) return attr;
+    ProfScope ps(kPDecodeAttn, st);
     decode_attn_kernel<64><<<agrid, 128, smem, st>>>(ap);
   }
   MSA_CHECK_LAUNCH();
@@ -550,8 +641,11 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   const int hpw = 32 / (p->d / 8);
   const int64_t warps = (int64_t(B) * p->g * R + hpw - 1) / hpw;
   const unsigned blocks = unsigned((warps + 7) / 8);
-  if (p->d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
-  else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
+  {
+    ProfScope ps(kPMerge, st);
+    if (p->d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
+    else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
+  }
   MSA_CHECK_LAUNCH();
   return MSA_OK;
 }
@@ -697,6 +791,49 @@ msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, cons
     return run_decode(p, q, k, v, q_idx, k_idx, block_ids_out, o, workspace, st);
   }
   return fail(MSA_ERR_INVALID_ARG, "mode=%d", p->mode);
+}
+
+msa_status_t msa_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = true;
+  return MSA_OK;
+}
+
+int32_t msa_profile_stop(msa_kernel_stat* out, int32_t max_out) {
+  std::vector<ProfRec> recs;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_on = false;
+    recs.swap(g_prof);
+  }
+  int launches[kPNumKinds] = {0};
+  double ms[kPNumKinds] = {0.0};
+  bool ok = true;
+  for (auto& r : recs) {
+    float t = 0.0f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) ok = false;
+    launches[r.kind] += 1;
+    ms[r.kind] += t;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto& r : recs) {
+      g_event_pool.push_back(r.a);
+      g_event_pool.push_back(r.b);
+    }
+  }
+  if (!ok) return -1;
+  int32_t n = 0;
+  for (int k = 0; k < kPNumKinds; ++k) {
+    if (launches[k] == 0) continue;
+    if (out && n < max_out) {
+      out[n].name = kProfNames[k];
+      out[n].launches = launches[k];
+      out[n].total_ms = ms[k];
+    }
+    ++n;
+  }
+  return n;
 }
 
 msa_status_t msa_get_device_error(void* stream) {

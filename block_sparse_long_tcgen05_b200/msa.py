@@ -22,7 +22,7 @@ MODE_PREFILL, MODE_DECODE = 0, 1
 # Every symbol include/msa.h declares.
 EXPORTS = ("msa_index_select_workspace", "msa_index_select", "msa_sparse_attn_workspace", "msa_sparse_attn",
            "msa_forward_workspace", "msa_forward", "msa_get_device_error", "msa_status_string",
-           "msa_last_error_detail")
+           "msa_last_error_detail", "msa_profile_start", "msa_profile_stop")
 
 
 class MsaError(RuntimeError):
@@ -36,6 +36,10 @@ class MsaParams(ctypes.Structure):
                 ("d", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("bk", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("scale", ctypes.c_float), ("n", ctypes.c_int64),
                 ("lmax", ctypes.c_int64), ("seqlens", ctypes.c_void_p), ("query_chunk", ctypes.c_int64)]
+
+
+class MsaKernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int32), ("total_ms", ctypes.c_double)]
 
 
 _lib = None
@@ -62,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_get_device_error": (c_i32, [c_p]),
         "msa_status_string": (ctypes.c_char_p, [c_i32]),
         "msa_last_error_detail": (ctypes.c_char_p, []),
+        "msa_profile_start": (c_i32, []),
+        "msa_profile_stop": (c_i32, [ctypes.POINTER(MsaKernelStat), c_i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -213,3 +219,18 @@ def check_device_error(device=None) -> None:
     st = msa_get_device_error(device)
     if st != MSA_OK:
         raise MsaError(st, load_library().msa_last_error_detail().decode())
+
+
+def msa_profile_start() -> None:
+    """Start recording CUDA events around every launch of the library."""
+    _check(load_library().msa_profile_start())
+
+
+def msa_profile_stop() -> dict:
+    """Stop recording; {kernel name: (launches, total device ms)} since msa_profile_start."""
+    lib = load_library()
+    buf = (MsaKernelStat * 32)()
+    n = lib.msa_profile_stop(buf, 32)
+    if n < 0:
+        raise MsaError(4, "profile events failed")
+    return {buf[i].name.decode(): (int(buf[i].launches), float(buf[i].total_ms)) for i in range(min(n, 32))}

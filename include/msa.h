@@ -120,6 +120,20 @@ MSA_API msa_status_t msa_forward(const msa_params* p, const void* q, const void*
  * last call), or MSA_ERR_CUDA when the synchronisation itself failed. */
 MSA_API msa_status_t msa_get_device_error(void* stream);
 
+/* Per-kernel timing (instrumentation for benchmarks; off by default).
+ * msa_profile_start() makes every later launch by this library, on any stream, record a
+ * CUDA event before and after itself. msa_profile_stop() waits for those events, stops
+ * recording and fills out[0 .. min(count, max_out)) with one entry per kernel kind that
+ * ran (name, launches, summed device milliseconds); it returns count, or -1 on a CUDA
+ * error. */
+typedef struct msa_kernel_stat {
+  const char* name;
+  int32_t launches;
+  double total_ms;
+} msa_kernel_stat;
+MSA_API msa_status_t msa_profile_start(void);
+MSA_API int32_t msa_profile_stop(msa_kernel_stat* out, int32_t max_out);
+
 /* Static English name of a status code. */
 MSA_API const char* msa_status_string(msa_status_t status);
 
