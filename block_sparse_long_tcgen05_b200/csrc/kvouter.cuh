@@ -314,59 +314,77 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           s = e & 31;
         }
         const int e_store = (storer && lane < nq) ? __ldg(P.entries + it.y + j * TQ + lane) : 0;
+        // warm L1 with the entries of this warpgroup's next tile (same item or the next one)
+        if (lane == 0) {
+          const int jn = j + 2;
+          const int32_t* pe = (jn < ntiles) ? P.entries + it.y + jn * TQ
+                                            : P.entries + nxt.y + (jn - ntiles) * TQ;
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(pe));
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(pe + TQ - 1));
+        }
         const int limit = !valid ? -1 : ((b == (i >> 7)) ? (i & 127) : 127);   // keys c <= limit are visible
         // warps whose rows all see the whole block skip the per-key mask
         const bool whole = __all_sync(0xffffffffu, limit == 127);
-        // ---- row max (pass 1 over S)
+        // ---- row max (pass 1 over S; two 32-column loads per TMEM wait)
         if (!fail && !mbar_wait(&s_full[wg], u & 1, abort_flag, kKidKvOuter)) fail = true;
         tc_fence_after();
         float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_s + c * 32, v);
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t v[2][32];
+          tmem_ld32(t_s + c * 32, v[0]);
+          tmem_ld32(t_s + c * 32 + 32, v[1]);
           tmem_ld_wait();
-          if (whole) {
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) mx = max3f(mx, __uint_as_float(v[x]), __uint_as_float(v[x + 1]));
-          } else {
+          for (int h = 0; h < 2; ++h) {
+            if (whole) {
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float a0 = (c * 32 + x <= limit) ? __uint_as_float(v[x]) : -INFINITY;
-              const float a1 = (c * 32 + x + 1 <= limit) ? __uint_as_float(v[x + 1]) : -INFINITY;
-              mx = max3f(mx, a0, a1);
+              for (int x = 0; x < 32; x += 2) mx = max3f(mx, __uint_as_float(v[h][x]), __uint_as_float(v[h][x + 1]));
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; x += 2) {
+                const int col = (c + h) * 32 + x;
+                const float a0 = (col <= limit) ? __uint_as_float(v[h][x]) : -INFINITY;
+                const float a1 = (col + 1 <= limit) ? __uint_as_float(v[h][x + 1]) : -INFINITY;
+                mx = max3f(mx, a0, a1);
+              }
             }
           }
         }
         const float mref = (limit >= 0) ? mx * P.scale_log2 : 0.0f;
         // ---- P = exp2(S * scale * log2e - max), written over S as bf16 (pass 2)
         float l = 0.0f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_s + c * 32, v);
+#pragma unroll 1
+        for (int c = 0; c < 4; c += 2) {
+          uint32_t v[2][32];
+          tmem_ld32(t_s + c * 32, v[0]);
+          tmem_ld32(t_s + c * 32 + 32, v[1]);
           tmem_ld_wait();
-          uint32_t pk[16];
-          if (whole) {
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float p0 = ex2_approx(fmaf(__uint_as_float(v[x]), P.scale_log2, -mref));
-              const float p1 = ex2_approx(fmaf(__uint_as_float(v[x + 1]), P.scale_log2, -mref));
-              l += p0 + p1;
-              pk[x >> 1] = pack_bf16x2(p0, p1);
-            }
-          } else {
+          for (int h = 0; h < 2; ++h) {
+            uint32_t pk[16];
+            if (whole) {
 #pragma unroll
-            for (int x = 0; x < 32; x += 2) {
-              const float p0 =
-                  (c * 32 + x <= limit) ? ex2_approx(fmaf(__uint_as_float(v[x]), P.scale_log2, -mref)) : 0.0f;
-              const float p1 =
-                  (c * 32 + x + 1 <= limit) ? ex2_approx(fmaf(__uint_as_float(v[x + 1]), P.scale_log2, -mref)) : 0.0f;
-              l += p0 + p1;
-              pk[x >> 1] = pack_bf16x2(p0, p1);
+              for (int x = 0; x < 32; x += 2) {
+                const float p0 = ex2_approx(fmaf(__uint_as_float(v[h][x]), P.scale_log2, -mref));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(v[h][x + 1]), P.scale_log2, -mref));
+                l += p0 + p1;
+                pk[x >> 1] = pack_bf16x2(p0, p1);
+              }
+            } else {
+#pragma unroll
+              for (int x = 0; x < 32; x += 2) {
+                const int col = (c + h) * 32 + x;
+                const float p0 =
+                    (col <= limit) ? ex2_approx(fmaf(__uint_as_float(v[h][x]), P.scale_log2, -mref)) : 0.0f;
+                const float p1 =
+                    (col + 1 <= limit) ? ex2_approx(fmaf(__uint_as_float(v[h][x + 1]), P.scale_log2, -mref)) : 0.0f;
+                l += p0 + p1;
+                pk[x >> 1] = pack_bf16x2(p0, p1);
+              }
             }
+            tmem_st16(t_s + (c + h) * 16, pk);
           }
-          tmem_st16(t_s + c * 16, pk);
         }
         tmem_st_wait();
         tc_fence_before();
@@ -378,20 +396,24 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
         if (storer) bulk_wait_read_all();            // this buffer's previous stores have read it
         named_bar_sync(bar_id, 128);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_o + c * 32, v);
+#pragma unroll 1
+        for (int c = 0; c < D / 32; c += 2) {
+          uint32_t v[2][32];
+          tmem_ld32(t_o + c * 32, v[0]);
+          tmem_ld32(t_o + c * 32 + 32, v[1]);
           tmem_ld_wait();
 #pragma unroll
-          for (int x = 0; x < 4; ++x) {              // four 16-byte chunks of 8 columns
-            const int ch = c * 4 + x;                // chunk index along d
-            const uint32_t addr = o_row + (ch >> 3) * 1024 + (((ch & 7) ^ (m & 7)) << 4);
-            st_shared_v4(addr,
-                         pack_bf16x2(__uint_as_float(v[x * 8 + 0]) * inv, __uint_as_float(v[x * 8 + 1]) * inv),
-                         pack_bf16x2(__uint_as_float(v[x * 8 + 2]) * inv, __uint_as_float(v[x * 8 + 3]) * inv),
-                         pack_bf16x2(__uint_as_float(v[x * 8 + 4]) * inv, __uint_as_float(v[x * 8 + 5]) * inv),
-                         pack_bf16x2(__uint_as_float(v[x * 8 + 6]) * inv, __uint_as_float(v[x * 8 + 7]) * inv));
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {              // four 16-byte chunks of 8 columns
+              const int ch = (c + h) * 4 + x;          // chunk index along d
+              const uint32_t addr = o_row + (ch >> 3) * 1024 + (((ch & 7) ^ (m & 7)) << 4);
+              const uint32_t* w = v[h] + x * 8;
+              st_shared_v4(addr, pack_bf16x2(__uint_as_float(w[0]) * inv, __uint_as_float(w[1]) * inv),
+                           pack_bf16x2(__uint_as_float(w[2]) * inv, __uint_as_float(w[3]) * inv),
+                           pack_bf16x2(__uint_as_float(w[4]) * inv, __uint_as_float(w[5]) * inv),
+                           pack_bf16x2(__uint_as_float(w[6]) * inv, __uint_as_float(w[7]) * inv));
+            }
           }
         }
         tc_fence_before();
