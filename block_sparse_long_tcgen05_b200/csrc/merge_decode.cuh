@@ -7,14 +7,17 @@
 namespace msa {
 
 // ------------------------------------------------------------------------------------
-// Merge: o[i, h] = sum_s exp(lse_s - L) * O_s, L = logsumexp_s lse_s, over the valid
-// slots of (i, g = h / R) in ascending slot order (deterministic). The partial O_s is
-// already normalised by its own softmax sum, so this is the exact softmax over the
-// union of the selected blocks (a fixed-order fp32 reduction; no atomics).
+// Merge. Slot s of (query i, group g) holds, per head, the unnormalised partial
+// O_s = sum_j 2^(x_j - m_s) v_j over the tokens of one selected block (x_j the logits in
+// log2 units), its row max m_s and row sum l_s = sum_j 2^(x_j - m_s). With M = max_s m_s
+// and w_s = 2^(m_s - M):
+//     o[i, h] = sum_s w_s O_s / sum_s w_s l_s,
+// which is exactly the softmax over the union of the selected blocks. Valid slots are
+// combined in ascending slot order (a fixed-order fp32 reduction; no atomics).
 // ------------------------------------------------------------------------------------
 struct MergeParams {
   const __nv_bfloat16* opart;  // [rows][G][k][R][D]
-  const float* lse;            // [rows][G][k][R]
+  const float2* ml;            // [rows][G][k][R]: (m_s, l_s)
   const int32_t* block_ids;    // [rows0 + rows][G][k] (absolute row index)
   __nv_bfloat16* o;            // [rows0 + rows][Hq][D]
   int64_t row0, rows;
@@ -38,19 +41,21 @@ __global__ void __launch_bounds__(256, 2) merge_kernel(const __grid_constant__ M
   const int64_t slot0 = (il * P.G + g) * P.k;
   const uint4* prow = reinterpret_cast<const uint4*>(P.opart + (slot0 * P.R + r) * D) + c;
   const int64_t pstride = static_cast<int64_t>(P.R) * D / 8;   // uint4 per slot
-  // The LPH lanes of this head row own slots c, c + LPH, ... for ids and lse. Every load of
-  // the row (ids, lse and the partials of the first 16 slots) is issued before any is
+  // The LPH lanes of this head row own slots c, c + LPH, ... for ids and (m, l). Every load
+  // of the row (ids, (m, l) and the partials of the first 16 slots) is issued before any is
   // used, so a row costs one memory round trip; slots past the valid ones are loaded but
   // never used (they hold no partial).
   const unsigned gmask = (LPH == 32) ? 0xffffffffu : (((1u << LPH) - 1u) << (lane & ~(LPH - 1)));
   const int lane0 = lane & ~(LPH - 1);
   int idv[4];
-  float own[4];
+  float own[4], lsum[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const int s = c + LPH * j;
     idv[j] = (s < P.k) ? __ldg(ids + s) : -1;
-    own[j] = (s < P.k) ? __ldg(P.lse + (slot0 + s) * P.R + r) : -INFINITY;
+    const float2 ml = (s < P.k) ? __ldg(P.ml + (slot0 + s) * P.R + r) : make_float2(-INFINITY, 0.0f);
+    own[j] = ml.x;
+    lsum[j] = ml.y;
   }
   uint4 raw[16];
 #pragma unroll
@@ -60,11 +65,11 @@ __global__ void __launch_bounds__(256, 2) merge_kernel(const __grid_constant__ M
   for (int j = 0; j < 4; ++j) nv += __popc(__ballot_sync(gmask, idv[j] >= 0) & gmask);
 #pragma unroll
   for (int j = 0; j < 4; ++j) own[j] = (c + LPH * j < nv) ? own[j] : -INFINITY;
-  float L = fmaxf(fmaxf(own[0], own[1]), fmaxf(own[2], own[3]));
+  float M = fmaxf(fmaxf(own[0], own[1]), fmaxf(own[2], own[3]));
 #pragma unroll
-  for (int o = 1; o < LPH; o <<= 1) L = fmaxf(L, __shfl_xor_sync(gmask, L, o));
+  for (int o = 1; o < LPH; o <<= 1) M = fmaxf(M, __shfl_xor_sync(gmask, M, o));
 #pragma unroll
-  for (int j = 0; j < 4; ++j) own[j] = (c + LPH * j < nv) ? __expf(own[j] - L) : 0.0f;
+  for (int j = 0; j < 4; ++j) own[j] = (c + LPH * j < nv) ? ex2_approx(own[j] - M) : 0.0f;
   float acc[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) acc[u] = 0.0f;
@@ -72,9 +77,11 @@ __global__ void __launch_bounds__(256, 2) merge_kernel(const __grid_constant__ M
   auto accumulate = [&](const uint4& rw, int s) {   // ascending slot order
     const int j = s / LPH;
     const float mine = (j == 0) ? own[0] : (j == 1) ? own[1] : (j == 2) ? own[2] : own[3];
+    const float myl = (j == 0) ? lsum[0] : (j == 1) ? lsum[1] : (j == 2) ? lsum[2] : lsum[3];
     const float wu = __shfl_sync(gmask, mine, lane0 + (s % LPH));
+    const float lu = __shfl_sync(gmask, myl, lane0 + (s % LPH));
     if (s < nv) {
-      W += wu;
+      W = fmaf(wu, lu, W);
       const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&rw);
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
@@ -193,8 +200,8 @@ __global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant_
 
 // ------------------------------------------------------------------------------------
 // Decode, Main Branch: one CTA per (sequence, group, slot): exact softmax attention of
-// the group's R heads over the slot's block (causal in the local block), written as a
-// normalised partial + lse for the merge kernel.
+// the group's R heads over the slot's block (causal in the local block), written as an
+// unnormalised partial with its (row max, row sum) for the merge kernel.
 // ------------------------------------------------------------------------------------
 struct DecodeAttnParams {
   const __nv_bfloat16* q;       // [B][Hq][D]
@@ -203,7 +210,7 @@ struct DecodeAttnParams {
   const int32_t* seqlens;
   const int32_t* block_ids;     // [B][G][k]
   __nv_bfloat16* opart;         // [B][G][k][R][D]
-  float* lse;                   // [B][G][k][R]
+  float2* ml;                   // [B][G][k][R]
   int B, G, R, k;
   int64_t Lmax;
   float scale_log2;
@@ -295,9 +302,9 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
     const int r = e / D, dd = e % D;
     float acc = 0.0f;
     for (int j = 0; j < nvalid; ++j) acc = fmaf(Ss[r * 128 + j], __bfloat162float(Vs[j * KS + dd]), acc);
-    P.opart[(slot * P.R + r) * D + dd] = __float2bfloat16_rn(acc / stat[2 * r + 1]);
+    P.opart[(slot * P.R + r) * D + dd] = __float2bfloat16_rn(acc);
   }
-  if (tid < P.R) P.lse[slot * P.R + tid] = (stat[2 * tid] + __log2f(stat[2 * tid + 1])) * 0.69314718055994531f;
+  if (tid < P.R) P.ml[slot * P.R + tid] = make_float2(stat[2 * tid], stat[2 * tid + 1]);
 }
 
 }  // namespace msa

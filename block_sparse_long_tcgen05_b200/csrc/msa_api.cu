@@ -369,7 +369,7 @@ struct AttnLayout {
   int32_t* entries = nullptr;
   int4* items = nullptr;
   void* opart = nullptr;
-  float* lse = nullptr;
+  float2* ml = nullptr;
   size_t bytes = 0;
 };
 
@@ -395,7 +395,7 @@ AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, in
   L.entries = static_cast<int32_t*>(cv.take(size_t(max_entries) * 4));
   L.items = static_cast<int4*>(cv.take(size_t(max_items) * 16));
   L.opart = cv.take(size_t(max_entries) * R * d * 2);
-  L.lse = static_cast<float*>(cv.take(size_t(max_entries) * R * 4));
+  L.ml = static_cast<float2*>(cv.take(size_t(max_entries) * R * 8));
   L.bytes = cv.off;
   return L;
 }
@@ -504,13 +504,13 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     kp.nbk = int(qa1);
     kp.row0 = qa0 * 128;
     kp.scale_log2 = scale * 1.4426950408889634f;
-    kp.lse = L.lse;
+    kp.ml = L.ml;
     if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, to, kp, st);
     else s = dispatch_kvouter<64>(R, tq, tk, tv, to, kp, st);
     if (s != MSA_OK) return s;
     MergeParams mp{};
     mp.opart = static_cast<const __nv_bfloat16*>(L.opart);
-    mp.lse = L.lse;
+    mp.ml = L.ml;
     mp.block_ids = block_ids;
     mp.o = static_cast<__nv_bfloat16*>(o);
     mp.row0 = qa0 * 128;
@@ -536,7 +536,7 @@ struct DecodeLayout {
   uint32_t* maxima = nullptr;
   int32_t* block_ids = nullptr;
   void* opart = nullptr;
-  float* lse = nullptr;
+  float2* ml = nullptr;
   size_t bytes = 0;
 };
 
@@ -549,7 +549,7 @@ DecodeLayout decode_layout(void* ws, const msa_params* p, bool need_ids) {
   L.maxima = static_cast<uint32_t*>(cv.take(size_t(B) * p->g * nbmax * 4));
   if (need_ids) L.block_ids = static_cast<int32_t*>(cv.take(size_t(B) * p->g * p->k * 4));
   L.opart = cv.take(size_t(B) * p->g * p->k * R * p->d * 2);
-  L.lse = static_cast<float*>(cv.take(size_t(B) * p->g * p->k * R * 4));
+  L.ml = static_cast<float2*>(cv.take(size_t(B) * p->g * p->k * R * 8));
   L.bytes = cv.off;
   return L;
 }
@@ -603,7 +603,7 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   ap.seqlens = p->seqlens;
   ap.block_ids = ids;
   ap.opart = static_cast<__nv_bfloat16*>(L.opart);
-  ap.lse = L.lse;
+  ap.ml = L.ml;
   ap.B = B;
   ap.G = p->g;
   ap.R = R;
@@ -630,7 +630,7 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   MSA_CHECK_LAUNCH();
   MergeParams mp{};
   mp.opart = static_cast<const __nv_bfloat16*>(L.opart);
-  mp.lse = L.lse;
+  mp.ml = L.ml;
   mp.block_ids = ids;
   mp.o = static_cast<__nv_bfloat16*>(o);
   mp.row0 = 0;
