@@ -72,7 +72,7 @@ int64_t tri(int64_t x) { return x * (x - 1) / 2; }
 size_t maxima_bytes(int64_t qb0, int64_t qb1, int G) { return size_t(4) * G * 128 * size_t(tri(qb1) - tri(qb0)); }
 
 // [qb0, qb1) ranges of the index branch
-std::vector<std::pair<int, int>> index_chunks(int64_t nb, int G) {
+std::vector<std::pair<int, int>> index_chunks(int64_t nb, int G, size_t cap = kMaximaCap) {
   std::vector<std::pair<int, int>> out;
   int64_t qb0 = 0;
   while (qb0 < nb) {
@@ -81,7 +81,7 @@ std::vector<std::pair<int, int>> index_chunks(int64_t nb, int G) {
     int64_t lo = qb0 + 1, hi = nb;
     while (lo < hi) {
       const int64_t mid = (lo + hi + 1) / 2;
-      if (maxima_bytes(qb0, mid, G) <= kMaximaCap && (mid + kIdxKbRun - 1) / kIdxKbRun <= kIdxMaxRuns) lo = mid;
+      if (maxima_bytes(qb0, mid, G) <= cap && (mid + kIdxKbRun - 1) / kIdxKbRun <= kIdxMaxRuns) lo = mid;
       else hi = mid - 1;
     }
     qb1 = lo;
@@ -226,6 +226,7 @@ struct ProfScope {
 struct IndexLayout {
   uint32_t* maxima = nullptr;
   size_t bytes = 0;
+  size_t cap = kMaximaCap;   // largest maxima buffer one index launch may fill
 };
 
 IndexLayout index_layout(void* ws, int64_t n, int32_t g) {
@@ -303,7 +304,7 @@ msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32
   if ((s = make_map_3d(&tq, q_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
   if ((s = make_map_3d(&tk, k_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
   const int sms = num_sms();
-  for (auto& ch : index_chunks(nb, g)) {
+  for (auto& ch : index_chunks(nb, g, L.cap)) {
     const int qb0 = ch.first, qb1 = ch.second;
     IdxParams P{};
     P.qb0 = qb0;
@@ -360,6 +361,38 @@ msa_status_t run_index_select(const void* q_idx, const void* k_idx, int64_t n, i
     case 128: return launch_index<128>(q_idx, k_idx, n, g, L, block_ids, k, st);
     default: return fail(MSA_ERR_UNSUPPORTED, "d_idx=%d", d_idx);
   }
+}
+
+// ------------------------ Index Branch without caller workspace ------------------------
+// Scratch for msa_index_select_static: the packed block maxima of one index launch live in
+// this file-scope device array instead of a caller-provided workspace. It is part of the
+// library's device image, so every GPU that loads the library holds it until the process
+// exits; calls on one device share it.
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+std::mutex g_static_mu;
+constexpr int kMaxDevices = 128;
+void* g_static_addr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once per device (host
+// code only sees a host-side stand-in for the symbol; that stand-in must never reach a
+// kernel). The first call on a device does the lookup.
+msa_status_t static_scratch_address(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MSA_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (g_static_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(MSA_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+    g_static_addr[dev] = p;
+  }
+  *out = g_static_addr[dev];
+  return MSA_OK;
 }
 
 // ------------------------------- main branch (prefill) -------------------------------
@@ -704,6 +737,38 @@ msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int64_t n, i
   if (workspace_bytes < need)
     return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
   return run_index_select(q_idx, k_idx, n, g, d_idx, k, block_ids, workspace, static_cast<cudaStream_t>(stream));
+}
+
+msa_status_t msa_index_select_static(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx,
+                                     int32_t bk, int32_t k, int32_t* block_ids, void* stream) {
+  g_detail[0] = 0;
+  msa_status_t s;
+  if ((s = check_common(n, g, bk, k)) != MSA_OK) return s;
+  if ((s = check_d_idx(d_idx)) != MSA_OK) return s;
+  if ((s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
+      (s = check_ptr(block_ids, "block_ids")) != MSA_OK)
+    return s;
+  // the launches are cut so that each fits the static scratch; the last query block alone
+  // needs 4 * g * 128 * (blocks - 1) bytes
+  const int64_t nb = (n + 127) / 128;
+  const size_t need = maxima_bytes(nb - 1, nb, g);
+  if (need > kStaticScratchBytes)
+    return fail(MSA_ERR_UNSUPPORTED,
+                "n=%lld with g=%d needs %zu bytes of block-maxima scratch per query block; the static scratch "
+                "holds %zu (use msa_index_select with a workspace)",
+                (long long)n, g, need, kStaticScratchBytes);
+  void* scratch = nullptr;
+  if ((s = static_scratch_address(&scratch)) != MSA_OK) return s;
+  IndexLayout L;
+  L.maxima = static_cast<uint32_t*>(scratch);
+  L.bytes = kStaticScratchBytes;
+  L.cap = kStaticScratchBytes;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (d_idx) {
+    case 32: return launch_index<32>(q_idx, k_idx, n, g, L, block_ids, k, st);
+    case 64: return launch_index<64>(q_idx, k_idx, n, g, L, block_ids, k, st);
+    default: return launch_index<128>(q_idx, k_idx, n, g, L, block_ids, k, st);
+  }
 }
 
 size_t msa_sparse_attn_workspace(int64_t n, int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t k) {

@@ -22,7 +22,7 @@ MODE_PREFILL, MODE_DECODE = 0, 1
 # Every symbol include/msa.h declares.
 EXPORTS = ("msa_index_select_workspace", "msa_index_select", "msa_sparse_attn_workspace", "msa_sparse_attn",
            "msa_forward_workspace", "msa_forward", "msa_get_device_error", "msa_status_string",
-           "msa_last_error_detail", "msa_profile_start", "msa_profile_stop")
+           "msa_last_error_detail", "msa_profile_start", "msa_profile_stop", "msa_index_select_static")
 
 
 class MsaError(RuntimeError):
@@ -68,6 +68,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_last_error_detail": (ctypes.c_char_p, []),
         "msa_profile_start": (c_i32, []),
         "msa_profile_stop": (c_i32, [ctypes.POINTER(MsaKernelStat), c_i32]),
+        "msa_index_select_static": (c_i32, [c_p, c_p, c_i64, c_i32, c_i32, c_i32, c_i32, c_p, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)

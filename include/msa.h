@@ -94,6 +94,27 @@ MSA_API msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int6
                               int32_t bk, int32_t k, int32_t* block_ids, void* workspace,
                               size_t workspace_bytes, void* stream);
 
+/* Index Branch for callers that cannot allocate device memory. This entry point has no
+ * counterpart in the method's description; it exists for callers that only hold a stream
+ * and raw tensor pointers, such as a plugin running inside another framework's execution
+ * engine or a serving loop that forbids device allocations after start-up, and so cannot
+ * call cudaMalloc to provide the workspace msa_index_select needs. It computes exactly what
+ * msa_index_select computes, with the same arguments minus the workspace.
+ *   Scratch: the block maxima live in a 32 MiB array inside the library's device image. Every
+ *   GPU that loads the library holds that array until the process exits. The query blocks
+ *   are processed in as many launches as it takes for each launch's maxima to fit; a problem
+ *   whose single last query block needs more than 32 MiB (4 * g * 128 * (ceil(n/128) - 1)
+ *   bytes) is rejected with MSA_ERR_UNSUPPORTED before anything is enqueued.
+ *   Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine is called.
+ *   The scratch needs no zeroing (every entry is written before it is read).
+ *   Set-up: the first call on a device looks up the array's device address (once per device,
+ *   with that device current); make that first call before any stream capture.
+ *   Calls on one device share the scratch: calls that overlap on the GPU (different streams,
+ *   or different host threads without ordering) race and give undefined results. */
+MSA_API msa_status_t msa_index_select_static(const void* q_idx, const void* k_idx, int64_t n, int32_t g,
+                                             int32_t d_idx, int32_t bk, int32_t k, int32_t* block_ids,
+                                             void* stream);
+
 /* Main Branch given the selection, executed KV-outer (each K/V block is held on chip
  * while the queries that chose it stream through; per-slot partial results are
  * merged by a deterministic log-sum-exp pass, no atomics).
