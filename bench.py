@@ -27,6 +27,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from block_sparse_long_tcgen05_b200 import accounting, synth  # noqa: E402
+from block_sparse_long_tcgen05_b200 import dist as mdist  # noqa: E402
 
 METRIC = "prefill tokens/s & TFLOP/s (frac of bf16 peak) at 128K; decode tokens/s"
 SPEC_BF16_TFLOPS = 2250.0
@@ -89,31 +90,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------------------------ dist
 def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
+    return mdist.init("nccl", timeout_s=300)
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return mdist.max_over_ranks(x, device="cuda") if world > 1 else x
 
 
 def barrier(world: int):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    mdist.barrier()
 
 
 # ------------------------------------------------------------------------------ CPU oracle
@@ -197,7 +182,7 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     peaks, peak_src = load_peaks()
     cfg = synth.CONFIGS[args.workload]
-    inp = synth.prefill_inputs(cfg, device=dev, seed=cfg.seed + 7 * rank)
+    inp = synth.prefill_inputs(cfg, device=dev, seed=mdist.rank_seed(cfg.seed, rank))
     N = cfg.N
     p = msa.prefill_params(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k)
     ws = torch.empty(msa.msa_forward_workspace(p), dtype=torch.uint8, device=dev)
@@ -273,7 +258,7 @@ def run_ours(args, world, rank, local):
     # ------------------------------------------------ decode (query-stationary), same ranks
     if not args.no_decode:
         dcfg = synth.DEC128K
-        dinp = synth.decode_inputs(dcfg, device=dev, seed=dcfg.seed + 7 * rank)
+        dinp = synth.decode_inputs(dcfg, device=dev, seed=mdist.rank_seed(dcfg.seed, rank))
         dp = msa.decode_params(dcfg.B, dinp["k_cache"].shape[1], dinp["seqlens"], dcfg.Hq, dcfg.G, dcfg.d,
                                dcfg.d_idx, dcfg.k)
         dws = torch.empty(msa.msa_forward_workspace(dp), dtype=torch.uint8, device=dev)
