@@ -1,0 +1,281 @@
+// Index Branch in one kernel: token scores, Block Max Pooling and the exp-free Top-k.
+//
+// hyper.ai "MiniMax Sparse Attention", Method (second paragraph): per GQA group, score every
+// visible key token with the dot product of the index query and the shared index key, pool
+// the scores to Bk = 128 blocks with a max, keep the Top-K blocks with the local block always
+// included; zhichai.net section 4.1: selection needs only the order of the scores, so no exp
+// is taken.
+//
+// Same tensor-core pipeline as index_blockmax (TMA -> tcgen05.mma M = 128 queries, N = 128
+// keys, K = d_idx -> TMEM, two query tiles per item sharing every key tile), but a work item
+// is a whole pair of query tiles {qa, qa + 1} of one group, over all its key blocks, so each
+// epilogue thread sees every block of its row: it keeps the best k - 1 keys
+// (ordkey(block max) << 32 | ~kb: higher score first, lower block index among equals) in
+// registers and writes the row's block_ids when the item ends. No block maxima reach memory.
+// Items are ordered group-major (one group's index keys, N * d_idx * 2 bytes, stay in L2
+// while all CTAs work on it), with the pairs of successive groups in alternating cost order,
+// and dealt to CTAs in snake order (alternating direction every round) so the per-CTA sums
+// of cost stay even.
+#pragma once
+#include "index_blockmax.cuh"
+#include "topk.cuh"
+
+namespace msa {
+
+struct IdxTopkParams {
+  int nb;              // query blocks of the sequence
+  int npairs;          // ceil(nb / 2)
+  int G, k;
+  int64_t N;
+  int32_t* block_ids;  // [N, G, k]
+};
+
+struct IdxTopkItem {
+  int g, qa, has_b, kbend;
+};
+
+// item t: group-major; within a group the pairs run in alternating directions (the last group
+// descending), so the cost of consecutive items never jumps and the list ends with the
+// cheapest items
+__device__ __forceinline__ IdxTopkItem idx_topk_item(const IdxTopkParams& P, int t) {
+  IdxTopkItem it;
+  it.g = t / P.npairs;
+  const int pr = t - it.g * P.npairs;
+  const int p = ((P.G - 1 - it.g) & 1) ? pr : P.npairs - 1 - pr;
+  it.qa = 2 * p;
+  it.has_b = (it.qa + 1 < P.nb) ? 1 : 0;
+  it.kbend = it.has_b ? it.qa + 1 : it.qa;
+  return it;
+}
+
+// CTA c's r-th item in snake order, or -1 when the round has none for it
+__device__ __forceinline__ int idx_topk_slot(int r, int total) {
+  const int grid = static_cast<int>(gridDim.x);
+  const int t = r * grid + ((r & 1) ? grid - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x));
+  return t < total ? t : -1;
+}
+
+template <int DI, int KM>
+__global__ void __launch_bounds__(kIdxThreads, 1)
+index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ IdxTopkParams P) {
+  using C = IdxCfg<DI>;
+  static_assert(KM >= 1, "at least one non-local place");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* q_full = bars + 0;              // [2]
+  uint64_t* q_empty = bars + 2;             // [2]
+  uint64_t* k_full = bars + 4;              // [stages]
+  uint64_t* k_empty = bars + 4 + kIdxStages;
+  uint64_t* acc_full = bars + 4 + 2 * kIdxStages;   // [2]
+  uint64_t* acc_empty = acc_full + 2;               // [2]
+  uint64_t* mma_done = acc_empty + 2;               // [1]
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+    for (int i = 0; i < kIdxStages; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_slot;
+  const int total = P.G * P.npairs;
+  const int rounds = (total + static_cast<int>(gridDim.x) - 1) / static_cast<int>(gridDim.x);
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      int64_t ik = 0;
+      int n_item = 0;
+      bool ok = true;
+      for (int r = 0; r < rounds && ok; ++r) {
+        const int t = idx_topk_slot(r, total);
+        if (t < 0) continue;
+        const IdxTopkItem it = idx_topk_item(P, t);
+        if (it.kbend == 0) continue;
+        const int qbuf = n_item & 1;
+        const uint32_t qu = static_cast<uint32_t>(n_item >> 1);
+        if (!mbar_wait(&q_empty[qbuf], (qu & 1) ^ 1, abort_flag, kKidIndexScore)) { ok = false; break; }
+        uint8_t* qa_s = smem + C::kQOff + (qbuf * 2 + 0) * C::kTileBytes;
+        uint8_t* qb_s = smem + C::kQOff + (qbuf * 2 + 1) * C::kTileBytes;
+        mbar_arrive_expect_tx(&q_full[qbuf], (it.has_b ? 2 : 1) * C::kTileBytes);
+        for (int pnl = 0; pnl < C::kPanels; ++pnl) {
+          tma_load_3d(qa_s + pnl * C::kPanelBytes, &tm_q, &q_full[qbuf], pnl * C::kPanelElems, it.g, it.qa * 128);
+          if (it.has_b)
+            tma_load_3d(qb_s + pnl * C::kPanelBytes, &tm_q, &q_full[qbuf], pnl * C::kPanelElems, it.g,
+                        (it.qa + 1) * 128);
+        }
+        ++n_item;
+        for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
+          const int s = static_cast<int>(ik % kIdxStages);
+          const uint32_t u = static_cast<uint32_t>(ik / kIdxStages);
+          if (!mbar_wait(&k_empty[s], (u & 1) ^ 1, abort_flag, kKidIndexScore)) { ok = false; break; }
+          uint8_t* ks = smem + C::kKOff + s * C::kTileBytes;
+          mbar_arrive_expect_tx(&k_full[s], C::kTileBytes);
+          for (int pnl = 0; pnl < C::kPanels; ++pnl)
+            tma_load_3d(ks + pnl * C::kPanelBytes, &tm_k, &k_full[s], pnl * C::kPanelElems, it.g, kb * 128);
+        }
+      }
+      // Drain: every TMA load this thread issued must land before the CTA exits.
+      for (int s = 0; s < kIdxStages; ++s) {
+        if (ik > s) {
+          const int64_t last = ((ik - 1 - s) / kIdxStages) * kIdxStages + s;
+          mbar_wait(&k_full[s], static_cast<uint32_t>(last / kIdxStages) & 1, nullptr, kKidIndexScore);
+        }
+      }
+      for (int b = 0; b < 2; ++b) {
+        if (n_item > b) {
+          const int last = ((n_item - 1 - b) / 2) * 2 + b;
+          mbar_wait(&q_full[b], static_cast<uint32_t>(last >> 1) & 1, nullptr, kKidIndexScore);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false);
+      int64_t ik = 0;
+      int n_item = 0;
+      bool ok = true;
+      for (int r = 0; r < rounds && ok; ++r) {
+        const int t = idx_topk_slot(r, total);
+        if (t < 0) continue;
+        const IdxTopkItem it = idx_topk_item(P, t);
+        if (it.kbend == 0) continue;
+        const int qbuf = n_item & 1;
+        const uint32_t qu = static_cast<uint32_t>(n_item >> 1);
+        ++n_item;
+        if (!mbar_wait(&q_full[qbuf], qu & 1, abort_flag, kKidIndexScore)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t qa_addr = smem_u32(smem + C::kQOff + (qbuf * 2 + 0) * C::kTileBytes);
+        const uint32_t qb_addr = smem_u32(smem + C::kQOff + (qbuf * 2 + 1) * C::kTileBytes);
+        for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
+          const int s = static_cast<int>(ik % kIdxStages);
+          const uint32_t u = static_cast<uint32_t>(ik / kIdxStages);
+          const int ab = static_cast<int>(ik & 1);
+          const uint32_t au = static_cast<uint32_t>(ik >> 1);
+          if (!mbar_wait(&k_full[s], u & 1, abort_flag, kKidIndexScore)) { ok = false; break; }
+          if (!mbar_wait(&acc_empty[ab], (au & 1) ^ 1, abort_flag, kKidIndexScore)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(smem + C::kKOff + s * C::kTileBytes);
+          const uint32_t d_a = tmem + ab * 256;
+          const uint32_t d_b = d_a + 128;
+          const bool a_active = kb < it.qa;
+#pragma unroll
+          for (int kk = 0; kk < C::kKSteps; ++kk) {
+            const uint32_t koff = (kk * 32) / C::kRowBytes * C::kPanelBytes + (kk * 32) % C::kRowBytes;
+            const uint64_t bdesc = smem_desc(k_addr + koff, 16, C::kSbo, C::kLayout);
+            if (a_active) umma_bf16(d_a, smem_desc(qa_addr + koff, 16, C::kSbo, C::kLayout), bdesc, idesc, kk > 0);
+            if (it.has_b) umma_bf16(d_b, smem_desc(qb_addr + koff, 16, C::kSbo, C::kLayout), bdesc, idesc, kk > 0);
+          }
+          umma_commit(&k_empty[s]);
+          umma_commit(&acc_full[ab]);
+        }
+        umma_commit(&q_empty[qbuf]);
+      }
+      umma_commit(mma_done);
+      mbar_wait(mma_done, 0, nullptr, kKidIndexScore);
+    }
+  } else {
+    // ------------------------------ epilogue: block max + running Top-k ------------------------------
+    const int ew = warp - 2;                 // 0..7
+    const int tile = ew >> 2;                // 0 = A (qa), 1 = B (qa + 1)
+    const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+    const int row = quad * 32 + lane;
+    int64_t ik = 0;
+    bool ok = true;
+    for (int r = 0; r < rounds && ok; ++r) {
+      const int t = idx_topk_slot(r, total);
+      if (t < 0) continue;
+      const IdxTopkItem it = idx_topk_item(P, t);
+      const int qb = it.qa + tile;
+      const bool tile_present = (tile == 0) || it.has_b;
+      uint64_t L[KM];
+#pragma unroll
+      for (int p = 0; p < KM; ++p) L[p] = 0ull;   // below every real key (ordered keys are > 0)
+      for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
+        const int ab = static_cast<int>(ik & 1);
+        const uint32_t au = static_cast<uint32_t>(ik >> 1);
+        if (!mbar_wait(&acc_full[ab], au & 1, abort_flag, kKidIndexScore)) { ok = false; break; }
+        tc_fence_after();
+        if (tile_present && kb < qb) {
+          const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + ab * 256 + tile * 128;
+          // the whole 128-column row in one TMEM round trip, then 8 independent max chains
+          uint32_t v[4][32];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, v[c]);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          float m8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) m8[j] = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int j = 0; j < 32; j += 2)
+              m8[(c * 16 + (j >> 1)) & 7] =
+                  max3f(m8[(c * 16 + (j >> 1)) & 7], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
+          float m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          m = __fadd_rn(m, 0.0f);   // -0 -> +0 so equal scores give equal keys
+          uint32_t u = __float_as_uint(m);
+          u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+          topk_insert<KM>(L, (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - kb));
+        } else {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+        }
+      }
+      if (!ok || !tile_present) continue;
+      const int64_t i = static_cast<int64_t>(qb) * 128 + row;
+      if (i >= P.N) continue;
+      int32_t* out = P.block_ids + (i * P.G + it.g) * P.k;
+      if (qb + 1 <= P.k) {
+        topk_all_visible(qb, P.k, out);
+      } else {
+        int ids[KM];
+#pragma unroll
+        for (int p = 0; p < KM; ++p) ids[p] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(L[p]));
+#pragma unroll
+        for (int pass = 0; pass < KM; ++pass) {
+#pragma unroll
+          for (int p = pass & 1; p + 1 < KM; p += 2) {
+            const int a = ids[p], b = ids[p + 1];
+            ids[p] = min(a, b);
+            ids[p + 1] = max(a, b);
+          }
+        }
+#pragma unroll
+        for (int p = 0; p < KM; ++p) out[p] = ids[p];
+        out[KM] = qb;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace msa

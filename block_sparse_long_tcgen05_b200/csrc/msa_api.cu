@@ -15,6 +15,7 @@
 #include "common.cuh"
 #include "csr.cuh"
 #include "index_blockmax.cuh"
+#include "index_topk.cuh"
 #include "kvouter.cuh"
 #include "merge_decode.cuh"
 #include "topk.cuh"
@@ -174,11 +175,11 @@ msa_status_t set_smem(K kernel, int bytes) {
 // ------------------------------- per-kernel timing -------------------------------
 enum ProfKind {
   kPIndex, kPTopkPrefill, kPCsrCount, kPCsrScan, kPCsrOffsets, kPCsrScatter, kPCsrItems, kPKvOuter, kPMerge,
-  kPDecodeScan, kPTopkDecode, kPDecodeAttn, kPNumKinds
+  kPDecodeScan, kPTopkDecode, kPDecodeAttn, kPIndexTopk, kPNumKinds
 };
 const char* const kProfNames[kPNumKinds] = {"index_blockmax", "topk_prefill", "csr_count", "csr_scan",
                                             "csr_offsets", "csr_scatter", "csr_items", "kvouter", "merge",
-                                            "decode_scan", "topk_decode", "decode_attn"};
+                                            "decode_scan", "topk_decode", "decode_attn", "index_topk"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -352,8 +353,69 @@ msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32
   return MSA_OK;
 }
 
+// The one-kernel Index Branch (Top-k fused into the score epilogue, no block maxima in
+// memory) serves the common k and sequences whose per-group index keys stay L2-resident
+// while every CTA streams them; anything else takes the two-kernel path.
+constexpr int64_t kFusedIndexMaxN = 262144;
+bool fused_index_ok(int64_t n, int32_t k) {
+  return n <= kFusedIndexMaxN && (k == 4 || k == 8 || k == 16 || k == 32);
+}
+
+size_t index_ws_bytes(int64_t n, int32_t g, int32_t k) {
+  return fused_index_ok(n, k) ? kAlign : index_layout(nullptr, n, g).bytes;
+}
+
+template <int DI, int KM>
+msa_status_t launch_index_topk_km(const CUtensorMap& tq, const CUtensorMap& tk, const IdxTopkParams& P,
+                                  cudaStream_t st) {
+  using C = IdxCfg<DI>;
+  static std::once_flag once;
+  static msa_status_t attr = MSA_OK;
+  std::call_once(once, [] { attr = set_smem(index_topk_kernel<DI, KM>, C::kSmemBytes); });
+  if (attr != MSA_OK) return attr;
+  const int total = P.G * P.npairs;
+  const int grid = std::min(num_sms(), total);
+  ProfScope ps(kPIndexTopk, st);
+  index_topk_kernel<DI, KM><<<grid, kIdxThreads, C::kSmemBytes, st>>>(tq, tk, P);
+  MSA_CHECK_LAUNCH();
+  return MSA_OK;
+}
+
+template <int DI>
+msa_status_t launch_index_topk(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t* block_ids,
+                               int32_t k, cudaStream_t st) {
+  using C = IdxCfg<DI>;
+  const uint64_t row_stride = uint64_t(g) * DI * 2;
+  CUtensorMap tq, tk;
+  const uint32_t box0 = C::kSw64 ? 32 : 64;
+  const CUtensorMapSwizzle sw = C::kSw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  msa_status_t s;
+  if ((s = make_map_3d(&tq, q_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
+  if ((s = make_map_3d(&tk, k_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
+  IdxTopkParams P{};
+  P.nb = int((n + 127) / 128);
+  P.npairs = (P.nb + 1) / 2;
+  P.G = g;
+  P.k = k;
+  P.N = n;
+  P.block_ids = block_ids;
+  switch (k) {
+    case 4: return launch_index_topk_km<DI, 3>(tq, tk, P, st);
+    case 8: return launch_index_topk_km<DI, 7>(tq, tk, P, st);
+    case 16: return launch_index_topk_km<DI, 15>(tq, tk, P, st);
+    default: return launch_index_topk_km<DI, 31>(tq, tk, P, st);
+  }
+}
+
 msa_status_t run_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx, int32_t k,
                               int32_t* block_ids, void* ws, cudaStream_t st) {
+  if (fused_index_ok(n, k)) {
+    switch (d_idx) {
+      case 32: return launch_index_topk<32>(q_idx, k_idx, n, g, block_ids, k, st);
+      case 64: return launch_index_topk<64>(q_idx, k_idx, n, g, block_ids, k, st);
+      default: return launch_index_topk<128>(q_idx, k_idx, n, g, block_ids, k, st);
+    }
+  }
   IndexLayout L = index_layout(ws, n, g);
   switch (d_idx) {
     case 32: return launch_index<32>(q_idx, k_idx, n, g, L, block_ids, k, st);
@@ -721,7 +783,7 @@ const char* msa_last_error_detail(void) { return g_detail; }
 
 size_t msa_index_select_workspace(int64_t n, int32_t g, int32_t d_idx, int32_t bk, int32_t k) {
   if (check_common(n, g, bk, k) != MSA_OK || check_d_idx(d_idx) != MSA_OK) return 0;
-  return index_layout(nullptr, n, g).bytes;
+  return index_ws_bytes(n, g, k);
 }
 
 msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx, int32_t bk,
@@ -733,7 +795,7 @@ msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int64_t n, i
   if ((s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
       (s = check_ptr(block_ids, "block_ids")) != MSA_OK || (s = check_ptr(workspace, "workspace")) != MSA_OK)
     return s;
-  const size_t need = index_layout(nullptr, n, g).bytes;
+  const size_t need = index_ws_bytes(n, g, k);
   if (workspace_bytes < need)
     return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
   return run_index_select(q_idx, k_idx, n, g, d_idx, k, block_ids, workspace, static_cast<cudaStream_t>(stream));
@@ -803,7 +865,7 @@ size_t msa_forward_workspace(const msa_params* p) {
       return 0;
     if (p->query_chunk < 0 || p->query_chunk % 128 != 0) return 0;
     const size_t a = attn_layout(nullptr, p->n, p->hq, p->g, p->d, p->k, p->query_chunk).bytes;
-    const size_t b = index_layout(nullptr, p->n, p->g).bytes;
+    const size_t b = index_ws_bytes(p->n, p->g, p->k);
     return prefill_ids_bytes(p->n, p->g, p->k) + std::max(a, b);
   }
   if (p->mode == MSA_MODE_DECODE) {

@@ -91,4 +91,9 @@ def test_workspace_sizes_grow_with_problem(lib):
     a = lib.msa_sparse_attn_workspace(32768, 64, 8, 128, 128, 16)
     b = lib.msa_sparse_attn_workspace(131072, 64, 8, 128, 128, 16)
     assert 0 < a <= b
-    assert lib.msa_index_select_workspace(131072, 8, 128, 128, 16) >= 4 * 8 * 128 * (1024 * 1023 // 2)
+    # k = 16 at 128K takes the one-kernel Index Branch: no block maxima in memory
+    assert 0 < lib.msa_index_select_workspace(131072, 8, 128, 128, 16) <= 4096
+    # k = 5 takes the two-kernel path: the packed maxima triangle lives in the workspace
+    assert lib.msa_index_select_workspace(131072, 8, 128, 128, 5) >= 4 * 8 * 128 * (1024 * 1023 // 2)
+    # beyond 256K tokens the two-kernel path is used for every k
+    assert lib.msa_index_select_workspace(524288, 8, 128, 128, 16) >= 4 * 8 * 128 * (4096 * 4095 // 2) // 8
