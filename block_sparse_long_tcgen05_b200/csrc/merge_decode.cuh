@@ -109,6 +109,157 @@ __global__ void __launch_bounds__(256, 2) merge_kernel(const __grid_constant__ M
 }
 
 // ------------------------------------------------------------------------------------
+// Streaming variant of the merge for the prefill chunks. One unit = one (query, group): its
+// k * R * D * 2-byte slab of partials is contiguous, so a producer warp brings it into a
+// ring of shared-memory stages with one bulk copy, and loads the unit's (m, l) pairs and
+// block ids into the same stage with plain loads; the consumer threads combine from shared
+// memory (same arithmetic and slot order as merge_kernel) and write o. Keeping several
+// stages in flight per SM is what lets this pass run at HBM bandwidth.
+// ------------------------------------------------------------------------------------
+constexpr int kMergeGroupThreads = 128;                  // one unit at a time per group
+constexpr int kMergeConsumers = 2 * kMergeGroupThreads;   // two groups on alternate units
+constexpr int kMergeThreads = 32 + kMergeConsumers;
+
+struct MergeStreamLayout {
+  int slab_bytes;   // k * R * D * 2
+  int ml_off;       // offset of the (m, l) pairs inside a stage
+  int ids_off;      // offset of the block ids
+  int stage_bytes;  // multiple of 128
+  int stages;
+  int bulk_meta;    // (m, l) and ids rows are 16-byte multiples: copy them in bulk too
+};
+
+template <int D>
+__global__ void __launch_bounds__(kMergeThreads, 1)
+merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant__ MergeStreamLayout S) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S.stages * S.stage_bytes);
+  uint64_t* empty = full + S.stages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S.stages);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S.stages; ++s) {
+      mbar_init(&full[s], 1 + 32);          // expect_tx arrival + one arrival per producer lane
+      mbar_init(&empty[s], kMergeGroupThreads / 32);   // the four warps of the unit's group
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int64_t units = P.rows * P.G;
+  const int64_t grid = gridDim.x;
+  const int kR = P.k * P.R;
+  if (warp == 0) {
+    // ---- producer: slab by bulk copy, (m, l) and ids by plain loads into the same stage
+    int n = 0;
+    for (int64_t u = blockIdx.x; u < units; u += grid, ++n) {
+      const int s = n % S.stages;
+      const uint32_t ph = static_cast<uint32_t>(n / S.stages);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(&empty[s], (ph & 1) ^ 1, abort_flag, kKidMerge) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      uint8_t* st = smem + s * S.stage_bytes;
+      const int64_t il = u / P.G, g = u % P.G;
+      const float2* mlsrc = P.ml + u * kR;
+      const int32_t* idsrc = P.block_ids + ((P.row0 + il) * P.G + g) * P.k;
+      if (lane == 0) {
+        // slab (and, when 16-byte aligned, the (m, l) pairs and ids) by bulk copy
+        mbar_arrive_expect_tx(&full[s], S.slab_bytes + (S.bulk_meta ? kR * 8 + P.k * 4 : 0));
+        bulk_load_g2s(st, P.opart + u * static_cast<int64_t>(kR) * D, S.slab_bytes, &full[s]);
+        if (S.bulk_meta) {
+          bulk_load_g2s(st + S.ml_off, mlsrc, kR * 8, &full[s]);
+          bulk_load_g2s(st + S.ids_off, idsrc, P.k * 4, &full[s]);
+        }
+      }
+      if (!S.bulk_meta) {
+        float2* mldst = reinterpret_cast<float2*>(st + S.ml_off);
+        for (int e = lane; e < kR; e += 32) mldst[e] = __ldg(mlsrc + e);
+        int32_t* iddst = reinterpret_cast<int32_t*>(st + S.ids_off);
+        for (int e = lane; e < P.k; e += 32) iddst[e] = __ldg(idsrc + e);
+      }
+      mbar_arrive(&full[s]);   // each lane: its stores above (if any) are released with this arrival
+    }
+    if (lane == 0 && n > 0) {   // drain the copies this warp issued
+      for (int s = 0; s < S.stages && s < n; ++s) {
+        const int last = ((n - 1 - s) / S.stages) * S.stages + s;
+        mbar_wait(&full[s], static_cast<uint32_t>(last / S.stages) & 1, nullptr, kKidMerge);
+      }
+    }
+  } else {
+    // ---- consumers: two groups of four warps take alternate units; within a unit, thread
+    // task (r, c) = head r, 16-byte chunk c of its D-wide row. Every slot's (m, l) and data
+    // are read from shared memory before any is combined (independent loads, one wait).
+    const int ct = threadIdx.x - 32;
+    const int grp = ct / kMergeGroupThreads;      // 0 or 1
+    const int gt = ct % kMergeGroupThreads;
+    constexpr int CPR = D / 8;
+    const int tasks = P.R * CPR;
+    const int Hq = P.G * P.R;
+    int n = 0;
+    for (int64_t u = blockIdx.x; u < units; u += grid, ++n) {
+      if ((n & 1) != grp) continue;
+      const int s = n % S.stages;
+      const uint32_t ph = static_cast<uint32_t>(n / S.stages);
+      if (!mbar_wait(&full[s], ph & 1, abort_flag, kKidMerge)) break;
+      const uint8_t* st = smem + s * S.stage_bytes;
+      const float2* ml = reinterpret_cast<const float2*>(st + S.ml_off);
+      const int32_t* ids = reinterpret_cast<const int32_t*>(st + S.ids_off);
+      int nv = 0;
+#pragma unroll 4
+      for (int x = 0; x < P.k; ++x) nv += (ids[x] >= 0) ? 1 : 0;   // valid ids come first
+      const int64_t i = P.row0 + u / P.G;
+      const int g = static_cast<int>(u % P.G);
+      for (int task = gt; task < tasks; task += kMergeGroupThreads) {
+        const int r = task / CPR, c = task % CPR;
+        float acc[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
+        float W = 0.0f;
+        float M4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // row max over the valid slots
+        for (int sl = 0; sl < nv; ++sl) M4[sl & 3] = fmaxf(M4[sl & 3], ml[sl * P.R + r].x);
+        const float M = fmaxf(fmaxf(M4[0], M4[1]), fmaxf(M4[2], M4[3]));
+        for (int s0 = 0; s0 < nv; s0 += 8) {   // batches of 8 slots, ascending
+          float2 mlv[8];
+          uint4 raw[8];
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            const int sl = s0 + x;
+            mlv[x] = (sl < nv) ? ml[sl * P.R + r] : make_float2(-INFINITY, 0.0f);
+            raw[x] = (sl < nv) ? *reinterpret_cast<const uint4*>(st + ((sl * P.R + r) * D + c * 8) * 2)
+                               : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int x = 0; x < 8; ++x) {
+            if (s0 + x < nv) {
+              const float w = ex2_approx(mlv[x].x - M);
+              W = fmaf(w, mlv[x].y, W);
+              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[x]);
+#pragma unroll
+              for (int t = 0; t < 4; ++t) {
+                const float2 f = __bfloat1622float2(h2[t]);
+                acc[2 * t] = fmaf(w, f.x, acc[2 * t]);
+                acc[2 * t + 1] = fmaf(w, f.y, acc[2 * t + 1]);
+              }
+            }
+          }
+        }
+        const float inv = (W > 0.0f) ? 1.0f / W : 0.0f;
+        uint4 out;
+        out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+        out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+        reinterpret_cast<uint4*>(P.o + (i * Hq + g * P.R + r) * D)[c] = out;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------------
 // Decode, Index Branch: block maxima of the one new query per sequence against every
 // full block before its local block (query-stationary: the index-key cache streams
 // through once, 64 contiguous bytes per lane per load).

@@ -516,6 +516,37 @@ msa_status_t dispatch_kvouter(int R, const CUtensorMap& tq, const CUtensorMap& t
   return launch_kvouter<D, 16>(tq, tk, tv, to, kp, st);
 }
 
+// The streaming merge: a ring of shared-memory stages, each holding one (query, group) slab
+// of partials plus its (m, l) pairs and ids; as many stages as fit ~200 KB, 2 at least.
+msa_status_t launch_merge_stream(const MergeParams& mp, int d, cudaStream_t st) {
+  MergeStreamLayout L{};
+  const int kR = mp.k * mp.R;
+  L.slab_bytes = kR * d * 2;
+  L.ml_off = (L.slab_bytes + 15) / 16 * 16;
+  L.ids_off = (L.ml_off + kR * 8 + 15) / 16 * 16;
+  L.stage_bytes = (L.ids_off + mp.k * 4 + 127) / 128 * 128;
+  L.stages = std::max(2, std::min(8, (200 * 1024) / L.stage_bytes));
+  L.bulk_meta = (kR % 2 == 0 && mp.k % 4 == 0) ? 1 : 0;
+  const int smem = L.stages * L.stage_bytes + L.stages * 16 + 16 + 128;
+  if (smem > 227 * 1024) return fail(MSA_ERR_UNSUPPORTED, "merge stage of %d bytes too large", L.stage_bytes);
+  static std::once_flag once;
+  static msa_status_t attr = MSA_OK;
+  std::call_once(once, [] {
+    attr = set_smem(merge_stream_kernel<128>, 227 * 1024);
+    if (attr == MSA_OK) attr = set_smem(merge_stream_kernel<64>, 227 * 1024);
+  });
+  if (attr != MSA_OK) return attr;
+  const int64_t units = mp.rows * mp.G;
+  const int grid = int(std::min<int64_t>(num_sms(), units));
+  {
+    ProfScope ps(kPMerge, st);
+    if (d == 128) merge_stream_kernel<128><<<grid, kMergeThreads, smem, st>>>(mp, L);
+    else merge_stream_kernel<64><<<grid, kMergeThreads, smem, st>>>(mp, L);
+  }
+  MSA_CHECK_LAUNCH();
+  return MSA_OK;
+}
+
 msa_status_t set_csr_smem() {
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
@@ -613,15 +644,7 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     mp.G = g;
     mp.R = R;
     mp.k = k;
-    const int hpw = 32 / (d / 8);
-    const int64_t warps = (mp.rows * g * R + hpw - 1) / hpw;
-    const unsigned blocks = unsigned((warps + 7) / 8);
-    {
-      ProfScope ps(kPMerge, st);
-      if (d == 128) merge_kernel<128><<<blocks, 256, 0, st>>>(mp);
-      else merge_kernel<64><<<blocks, 256, 0, st>>>(mp);
-    }
-    MSA_CHECK_LAUNCH();
+    if ((s = launch_merge_stream(mp, d, st)) != MSA_OK) return s;
   }
   return MSA_OK;
 }
