@@ -17,18 +17,21 @@
 //   the k slots of every query (no atomics).
 //
 // Roles (16 warps):
-//   warp 0        TMA loads of K_b and V_b
-//   warp 1        tcgen05.mma issue (a ready PV goes before the next S)
+//   warp 0        TMA loads of K_b and V_b (two buffers each: the next item's block loads
+//                 while the current one is still in use)
+//   warp 1        tcgen05.mma issue of S = Q K^T, in tile order
 //   warp 2        TMA gather of query rows (one 2 KB box per 8 rows: both 64-column panels)
-//   warp 3        TMA stores of the staged partials
+//   warp 3        tcgen05.mma issue of O = P V, in tile order. Two issuers, because an issue
+//                 sequence stalls while the tensor pipe is busy: a PV that is ready does not
+//                 wait behind the S product of the next tile, nor the other way round.
 //   warps 4..7    softmax warpgroup 0 (tiles with even index)
 //   warps 8..11   softmax warpgroup 1 (odd tiles): the two alternate on the exp unit
-//   warps 12..15  epilogue warpgroup: O from TMEM to bf16 staging, for every tile
-// Tile n uses TMEM pair w = n % 2 (S/P at column 128*w, O at 256 + 128*w) and staging w.
+//   warps 12..15  epilogue warpgroup: O from TMEM to bf16, stored straight to the partials
+// Tile n uses TMEM pair w = n % 2 (S/P at column 128*w, O at 256 + 128*w).
 //
 // Shared-memory layouts (all 128-byte swizzled, 1024-byte aligned):
 //   K, V: [panel][128 keys][128 B]                     (8-row group stride 1 KB, panel 16 KB)
-//   Q, staging: [8-row group][panel][8 rows][128 B]    (8-row group stride kPanels KB, panel 1 KB)
+//   Q: [8-row group][panel][8 rows][128 B]             (8-row group stride kPanels KB, panel 1 KB)
 #pragma once
 #include "ptx.cuh"
 
@@ -44,11 +47,10 @@ struct KvCfg {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kGroupBytes = kPanels * 1024;     // one 8-row group, all panels
   static constexpr int TQ = 128 / RP;
-  static constexpr int kKOff = 0;
-  static constexpr int kVOff = kTileBytes;
-  static constexpr int kQOff = 2 * kTileBytes;
-  static constexpr int kOOff = kQOff + kKvQStages * kTileBytes;   // 2 staging buffers
-  static constexpr int kBarOff = kOOff + 2 * kTileBytes;
+  static constexpr int kKOff = 0;                        // 2 K buffers
+  static constexpr int kVOff = 2 * kTileBytes;           // 2 V buffers
+  static constexpr int kQOff = 4 * kTileBytes;           // kKvQStages query stages
+  static constexpr int kBarOff = kQOff + kKvQStages * kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
@@ -60,52 +62,51 @@ struct KvParams {
   int64_t row0;              // first query of the chunk
   float scale_log2;
   float2* ml;                // [chunk rows][G][k][R]: (row max in log2 units, row sum)
+  uint16_t* opart;           // [chunk rows][G][k][R][D] bf16: unnormalised partial outputs
 };
 
 // tensor maps:
 //   tm_q: 4-D view of q [N][Hq][D] as (64 elems, Hq heads, D/64 panels, N), box (64, 8, D/64, 1)
 //   tm_k, tm_v: 3-D view of k / v [N][G][D] as (D, G, N), box (64, 1, 128)
-//   tm_o: 4-D view of the partials [rows][R][D] as (64, R, D/64, rows),
-//         box (64, min(R, 8), R >= 8 ? D/64 : 1, 1)
 template <int D, int RP>
 __global__ void __launch_bounds__(kKvThreads, 1)
 kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-               const __grid_constant__ KvParams P) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ KvParams P) {
   using C = KvCfg<D, RP>;
   constexpr int TQ = C::TQ;
   constexpr int QS = kKvQStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* k_full = bars + 0;
-  uint64_t* k_empty = bars + 1;
-  uint64_t* v_full = bars + 2;
-  uint64_t* v_empty = bars + 3;
-  uint64_t* q_full = bars + 4;              // [QS]
-  uint64_t* q_empty = bars + 4 + QS;        // [QS]
-  uint64_t* s_full = bars + 4 + 2 * QS;     // [2] S of tile n in TMEM (MMA -> softmax)
-  uint64_t* p_full = s_full + 2;            // [2] P written over S (softmax, 4 warps -> MMA)
-  uint64_t* o_full = s_full + 4;            // [2] PV done (MMA -> epilogue; also frees S/P)
-  uint64_t* o_free = s_full + 6;            // [2] O read out (epilogue, 4 warps -> MMA)
-  uint64_t* stg_full = s_full + 8;          // [2] staging written (epilogue, 4 warps -> store warp)
-  uint64_t* stg_empty = s_full + 10;        // [2] staging read by its TMA stores (store warp -> epilogue)
-  uint64_t* mma_done = s_full + 12;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* k_full = bars + 0;              // [2] per K buffer
+  uint64_t* k_empty = bars + 2;             // [2]
+  uint64_t* v_full = bars + 4;              // [2] per V buffer
+  uint64_t* v_empty = bars + 6;             // [2]
+  uint64_t* q_full = bars + 8;              // [QS]
+  uint64_t* q_empty = bars + 8 + QS;        // [QS]
+  uint64_t* s_full = bars + 8 + 2 * QS;     // [2] S of tile n in TMEM (S issuer -> softmax)
+  uint64_t* p_full = s_full + 2;            // [2] P written over S (softmax, 4 warps -> PV issuer)
+  uint64_t* o_full = s_full + 4;            // [2] PV done (PV issuer -> epilogue; also frees S/P)
+  uint64_t* o_free = s_full + 6;            // [2] O read out (epilogue, 4 warps -> PV issuer)
+  uint64_t* s_done = s_full + 8;            // all S products of the CTA complete
+  uint64_t* pv_done = s_full + 9;           // all PV products of the CTA complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(k_full, 1); mbar_init(k_empty, 1); mbar_init(v_full, 1); mbar_init(v_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
+    }
     for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4);
       mbar_init(&o_full[i], 1); mbar_init(&o_free[i], 4);
-      mbar_init(&stg_full[i], 4); mbar_init(&stg_empty[i], 1);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(s_done, 1);
+    mbar_init(pv_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -123,6 +124,8 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   if (warp == 0) {
     // ------------------------------ K / V producer ------------------------------
+    // Item ni uses K / V buffer ni % 2; a buffer is refilled once the last S (for K) or
+    // PV (for V) product of the item before the previous one has completed.
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -132,20 +135,24 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int4 it = nxt;
         if (t + grid < n_items) nxt = P.items[t + grid];
         const int g = it.x / P.nbk, b = it.x % P.nbk;
-        if (!mbar_wait(k_empty, (ni & 1) ^ 1, abort_flag, kKidKvOuter)) break;
-        mbar_arrive_expect_tx(k_full, C::kTileBytes);
+        const int kb = ni & 1;
+        const uint32_t ph = static_cast<uint32_t>(ni >> 1) & 1;
+        if (!mbar_wait(&k_empty[kb], ph ^ 1, abort_flag, kKidKvOuter)) break;
+        mbar_arrive_expect_tx(&k_full[kb], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(smem + C::kKOff + p * 16384, &tm_k, k_full, p * 64, g, b * 128);
+          tma_load_3d(smem + C::kKOff + kb * C::kTileBytes + p * 16384, &tm_k, &k_full[kb], p * 64, g, b * 128);
         ++kn;
-        if (!mbar_wait(v_empty, (ni & 1) ^ 1, abort_flag, kKidKvOuter)) break;
-        mbar_arrive_expect_tx(v_full, C::kTileBytes);
+        if (!mbar_wait(&v_empty[kb], ph ^ 1, abort_flag, kKidKvOuter)) break;
+        mbar_arrive_expect_tx(&v_full[kb], C::kTileBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(smem + C::kVOff + p * 16384, &tm_v, v_full, p * 64, g, b * 128);
+          tma_load_3d(smem + C::kVOff + kb * C::kTileBytes + p * 16384, &tm_v, &v_full[kb], p * 64, g, b * 128);
         ++vn;
       }
-      // drain: the last K and V loads issued must land before the CTA exits
-      if (kn > 0) mbar_wait(k_full, (kn - 1) & 1, nullptr, kKidKvOuter);
-      if (vn > 0) mbar_wait(v_full, (vn - 1) & 1, nullptr, kKidKvOuter);
+      // drain: the last K and V loads issued into each buffer must land before the CTA exits
+      for (int x = 1; x <= 2; ++x) {
+        if (kn >= x) mbar_wait(&k_full[(kn - x) & 1], static_cast<uint32_t>((kn - x) >> 1) & 1, nullptr, kKidKvOuter);
+        if (vn >= x) mbar_wait(&v_full[(vn - x) & 1], static_cast<uint32_t>((vn - x) >> 1) & 1, nullptr, kKidKvOuter);
+      }
     }
   } else if (warp == 2) {
     // ------------------------------ query gather ------------------------------
@@ -187,64 +194,38 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
-    // Event loop over two cursors of this CTA's tile sequence: PV(n) as soon as P(n) is
-    // written (it ends warpgroup n%2's cycle), otherwise S(n) as soon as its query rows are
-    // loaded and PV(n - 2), which read P from the same TMEM columns, has completed.
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------ MMA issuers ------------------------------
+    // warp 1: S(n) once its query rows and its item's K are in shared memory and PV(n - 2),
+    //         which read P from the same TMEM columns, has completed.
+    // warp 3: PV(n) once P(n) is written, its item's V is in shared memory and the epilogue
+    //         has read O(n - 2) out of the same TMEM columns.
     if (lane == 0) {
+      const bool is_s = (warp == 1);
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
-      const uint32_t k_addr = smem_u32(smem + C::kKOff);
-      const uint32_t v_addr = smem_u32(smem + C::kVOff);
-      struct Cursor {
-        int t, j, ntiles, n, ni;
-      };
-      auto start = [&](Cursor& c) {
-        c.t = blockIdx.x; c.j = 0; c.n = 0; c.ni = 0;
-        c.ntiles = (c.t < n_items) ? (first_item.z + TQ - 1) / TQ : 0;
-      };
-      auto advance = [&](Cursor& c) {
-        ++c.n;
-        if (++c.j == c.ntiles) {
-          c.j = 0;
-          c.t += grid;
-          ++c.ni;
-          c.ntiles = (c.t < n_items) ? (__ldg(&P.items[c.t].z) + TQ - 1) / TQ : 0;
-        }
-      };
-      Cursor cs, cp;   // next S to issue, next PV to issue
-      start(cs);
-      start(cp);
-      uint64_t idle_since = 0;
+      int n = 0, ni = 0;
       bool ok = true;
-      while (ok && (cs.t < n_items || cp.n < cs.n)) {
-        bool progressed = false;
-        if (cp.n < cs.n) {
-          const int w = cp.n & 1;
-          const uint32_t u = static_cast<uint32_t>(cp.n >> 1);
-          if ((cp.j != 0 || mbar_test(v_full, cp.ni & 1)) && mbar_test(&p_full[w], u & 1) &&
-              mbar_test(&o_free[w], (u & 1) ^ 1)) {
-            tc_fence_after();
-            const uint32_t d_o = tmem + 256 + w * 128;
-            const uint32_t a_p = tmem + w * 128;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(v_addr + kk * 2048, 16384, 1024, kLayoutSw128), idesc_o,
-                           kk > 0);
-            umma_commit(&o_full[w]);
-            if (cp.j == cp.ntiles - 1) umma_commit(v_empty);
-            advance(cp);
-            progressed = true;
-          }
-        }
-        if (!progressed && cs.t < n_items) {
-          const int qs = cs.n % QS;
-          const int w = cs.n & 1;
-          const uint32_t u = static_cast<uint32_t>(cs.n >> 1);
-          if ((cs.j != 0 || mbar_test(k_full, cs.ni & 1)) &&
-              mbar_test(&q_full[qs], static_cast<uint32_t>(cs.n / QS) & 1) &&
-              mbar_test(&o_full[w], (u & 1) ^ 1)) {
+      int4 nxt = first_item;
+      for (int t = blockIdx.x; t < n_items && ok; t += grid, ++ni) {
+        const int4 it = nxt;
+        if (t + grid < n_items) nxt = P.items[t + grid];
+        const int ntiles = (it.z + TQ - 1) / TQ;
+        const int kb = ni & 1;
+        const uint32_t ph = static_cast<uint32_t>(ni >> 1) & 1;
+        const uint32_t k_addr = smem_u32(smem + C::kKOff + kb * C::kTileBytes);
+        const uint32_t v_addr = smem_u32(smem + C::kVOff + kb * C::kTileBytes);
+        if (!mbar_wait(is_s ? &k_full[kb] : &v_full[kb], ph, abort_flag, kKidKvOuter)) { ok = false; break; }
+        for (int j = 0; j < ntiles; ++j, ++n) {
+          const int w = n & 1;
+          const uint32_t u = static_cast<uint32_t>(n >> 1);
+          if (is_s) {
+            const int qs = n % QS;
+            if (!mbar_wait(&q_full[qs], static_cast<uint32_t>(n / QS) & 1, abort_flag, kKidKvOuter) ||
+                !mbar_wait(&o_full[w], (u & 1) ^ 1, abort_flag, kKidKvOuter)) {
+              ok = false;
+              break;
+            }
             tc_fence_after();
             const uint32_t q_addr = smem_u32(smem + C::kQOff + qs * C::kTileBytes);
             const uint32_t d_s = tmem + w * 128;
@@ -257,38 +238,44 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             umma_commit(&q_empty[qs]);
             umma_commit(&s_full[w]);
-            if (cs.j == cs.ntiles - 1) umma_commit(k_empty);
-            advance(cs);
-            progressed = true;
+            if (j == ntiles - 1) umma_commit(&k_empty[kb]);
+          } else {
+            if (!mbar_wait(&p_full[w], u & 1, abort_flag, kKidKvOuter) ||
+                !mbar_wait(&o_free[w], (u & 1) ^ 1, abort_flag, kKidKvOuter)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d_o = tmem + 256 + w * 128;
+            const uint32_t a_p = tmem + w * 128;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(v_addr + kk * 2048, 16384, 1024, kLayoutSw128), idesc_o,
+                           kk > 0);
+            umma_commit(&o_full[w]);
+            if (j == ntiles - 1) umma_commit(&v_empty[kb]);
           }
-        }
-        if (progressed) {
-          idle_since = 0;
-        } else {
-          // bounded idling: give up (and make every role give up) after the wait limit
-          const uint64_t now = globaltimer_ns();
-          if (idle_since == 0) idle_since = now;
-          if (*abort_flag) ok = false;
-          else if (now - idle_since > kWaitLimitNs) {
-            record_error(MSA_ERR_TIMEOUT, kKidKvOuter);
-            *abort_flag = 1;
-            ok = false;
-          }
-          __nanosleep(20);
         }
       }
-      umma_commit(mma_done);
-      mbar_wait(mma_done, 0, nullptr, kKidKvOuter);
+      // every product this thread issued completes before TMEM is released
+      uint64_t* done = is_s ? s_done : pv_done;
+      umma_commit(done);
+      mbar_wait(done, 0, nullptr, kKidKvOuter);
     }
-  } else if (warp == 3) {
-    // ------------------------------ partial stores ------------------------------
-    // Once the epilogue warps have staged a tile, lane q issues query q's TMA stores; when
-    // every store has read the staging buffer, it is handed back.
-    if (lane == 0) tma_prefetch_desc(&tm_o);
+  } else if (warp >= 12) {
+    // ------------------------------ epilogue warpgroup ------------------------------
+    // O of every tile: TMEM -> bf16 -> the partial row of (query, slot, head), one 32-byte
+    // store per 16 columns. The TMEM columns are handed back as soon as the last load has
+    // landed; the stores follow from registers.
+    const int quad = warp & 3;
+    const int m = quad * 32 + lane;
+    const int q = m / RP, r = m % RP;
+    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
+    const uint64_t policy = l2_policy_evict_first();
     int nt = 0;
-    bool ok = true;
+    bool fail = false;
     int4 nxt = first_item;
-    for (int t = blockIdx.x; t < n_items && ok; t += grid) {
+    for (int t = blockIdx.x; t < n_items && !fail; t += grid) {
       const int4 it = nxt;
       if (t + grid < n_items) nxt = P.items[t + grid];
       const int g = it.x / P.nbk;
@@ -297,84 +284,39 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int w = nt & 1;
         const uint32_t u = static_cast<uint32_t>(nt >> 1);
         const int nq = min(TQ, it.z - j * TQ);
-        const int e = (lane < nq) ? __ldg(P.entries + it.y + j * TQ + lane) : 0;
-        int w_ok = 1;
-        if (lane == 0) w_ok = mbar_wait(&stg_full[w], u & 1, abort_flag, kKidKvOuter) ? 1 : 0;
-        w_ok = __shfl_sync(0xffffffffu, w_ok, 0);
-        if (!w_ok) { ok = false; break; }
-        if (lane < nq) {
-          const int64_t il = static_cast<int64_t>(e >> 5) - P.row0;
-          const int row = static_cast<int>((il * P.G + g) * P.k + (e & 31));
-          const uint8_t* src = smem + C::kOOff + w * C::kTileBytes + lane * (RP / 8) * C::kGroupBytes;
-          if (P.R >= 8) {
-#pragma unroll
-            for (int h8 = 0; h8 < RP / 8; ++h8) tma_store_4d(&tm_o, src + h8 * C::kGroupBytes, 0, h8 * 8, 0, row);
-          } else {
-#pragma unroll
-            for (int p = 0; p < C::kPanels; ++p) tma_store_4d(&tm_o, src + p * 1024, 0, 0, p, row);
-          }
-          bulk_commit_group();
-          bulk_wait_read_all();
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&stg_empty[w]);
-      }
-    }
-    bulk_wait_all();
-  } else if (warp >= 12) {
-    // ------------------------------ epilogue warpgroup ------------------------------
-    // O of every tile: TMEM -> bf16 -> swizzled staging, then handed to the store warp.
-    const int quad = warp & 3;
-    const int m = quad * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    int nt = 0;
-    bool fail = false;
-    int4 nxt = first_item;
-    for (int t = blockIdx.x; t < n_items && !fail; t += grid) {
-      const int4 it = nxt;
-      if (t + grid < n_items) nxt = P.items[t + grid];
-      const int ntiles = (it.z + TQ - 1) / TQ;
-      for (int j = 0; j < ntiles; ++j, ++nt) {
-        const int w = nt & 1;
-        const uint32_t u = static_cast<uint32_t>(nt >> 1);
+        const bool valid = (q < nq) && (r < P.R);
+        const int e = valid ? __ldg(P.entries + it.y + j * TQ + q) : 0;
         const uint32_t t_o = tmem + lane_base + 256 + w * 128;
-        const uint32_t o_row = smem_u32(smem + C::kOOff + w * C::kTileBytes) + (m >> 3) * C::kGroupBytes + (m & 7) * 128;
         if (!mbar_wait(&o_full[w], u & 1, abort_flag, kKidKvOuter)) { fail = true; break; }
-        if (!mbar_wait(&stg_empty[w], (u & 1) ^ 1, abort_flag, kKidKvOuter)) { fail = true; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < D / 32; c += 2) {
+        uint32_t pk[D / 2];
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t v[2][32];
-          tmem_ld32(t_o + c * 32, v[0]);
-          tmem_ld32(t_o + c * 32 + 32, v[1]);
+          tmem_ld32(t_o + c * 64, v[0]);
+          tmem_ld32(t_o + c * 64 + 32, v[1]);
           tmem_ld_wait();
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {              // four 16-byte chunks of 8 columns
-              const int ch = (c + h) * 4 + x;          // chunk index along d
-              const uint32_t addr = o_row + (ch >> 3) * 1024 + (((ch & 7) ^ (m & 7)) << 4);
-              const uint32_t* s8 = v[h] + x * 8;
-              st_shared_v4(addr, pack_bf16x2(__uint_as_float(s8[0]), __uint_as_float(s8[1])),
-                           pack_bf16x2(__uint_as_float(s8[2]), __uint_as_float(s8[3])),
-                           pack_bf16x2(__uint_as_float(s8[4]), __uint_as_float(s8[5])),
-                           pack_bf16x2(__uint_as_float(s8[6]), __uint_as_float(s8[7])));
-            }
+          if (c == D / 64 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[w]);
           }
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            pk[c * 32 + x] = pack_bf16x2(__uint_as_float(v[x >> 4][(2 * x) & 31]), __uint_as_float(v[x >> 4][(2 * x + 1) & 31]));
         }
-        tc_fence_before();
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&o_free[w]);
-          mbar_arrive(&stg_full[w]);
+        if (valid) {
+          const int64_t il = static_cast<int64_t>(e >> 5) - P.row0;
+          uint16_t* dst = P.opart + (((il * P.G + g) * P.k + (e & 31)) * P.R + r) * D;
+#pragma unroll
+          for (int z = 0; z < D / 16; ++z) st_global_v8(dst + z * 16, pk + z * 8, policy);
         }
       }
     }
   } else if (warp >= 4) {
     // ------------------------------ softmax warpgroups ------------------------------
     // The four warps of a warpgroup never wait for one another: each hands its rows over
-    // through mbarrier arrivals (P to the MMA warp).
+    // through mbarrier arrivals (P to the PV issuer).
     const int wg = (warp - 4) >> 2;               // 0 or 1: takes tiles with nt % 2 == wg
     const int quad = warp & 3;
     const int m = quad * 32 + lane;               // row of the tile == TMEM lane

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -67,6 +68,7 @@ constexpr int64_t kMaxN = (int64_t(1) << 26) - 1;
 // ranges whose packed block maxima fit this cap.
 constexpr size_t kMaximaCap = size_t(4) << 30;
 constexpr int64_t kDefaultQueryChunk = 16384;
+constexpr int kDefaultMergeSms = 0;
 
 int64_t tri(int64_t x) { return x * (x - 1) / 2; }
 
@@ -460,11 +462,12 @@ msa_status_t static_scratch_address(void** out) {
 // ------------------------------- main branch (prefill) -------------------------------
 struct AttnLayout {
   int64_t chunk_blocks = 0;   // query blocks per chunk
+  int64_t chunks = 0;
   uint32_t *hist = nullptr, *totals = nullptr, *bstart = nullptr, *istart = nullptr;
   int32_t* entries = nullptr;
   int4* items = nullptr;
-  void* opart = nullptr;
-  float2* ml = nullptr;
+  void* opart[2] = {nullptr, nullptr};   // chunk c uses buffer c % 2 (one buffer for one chunk)
+  float2* ml[2] = {nullptr, nullptr};
   size_t bytes = 0;
 };
 
@@ -478,6 +481,7 @@ AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, in
   cq = std::max<int64_t>(1, std::min(cq, nb));
   AttnLayout L;
   L.chunk_blocks = cq;
+  L.chunks = (nb + cq - 1) / cq;
   const int64_t rows = cq * 128;
   const int64_t nbuck = int64_t(g) * nb;
   const int64_t max_entries = rows * g * k;
@@ -489,36 +493,40 @@ AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, in
   L.istart = static_cast<uint32_t*>(cv.take(size_t(nbuck + 1) * 4));
   L.entries = static_cast<int32_t*>(cv.take(size_t(max_entries) * 4));
   L.items = static_cast<int4*>(cv.take(size_t(max_items) * 16));
-  L.opart = cv.take(size_t(max_entries) * R * d * 2);
-  L.ml = static_cast<float2*>(cv.take(size_t(max_entries) * R * 8));
+  const int nbuf = L.chunks > 1 ? 2 : 1;
+  for (int i = 0; i < nbuf; ++i) {
+    L.opart[i] = cv.take(size_t(max_entries) * R * d * 2);
+    L.ml[i] = static_cast<float2*>(cv.take(size_t(max_entries) * R * 8));
+  }
+  if (nbuf == 1) { L.opart[1] = L.opart[0]; L.ml[1] = L.ml[0]; }
   L.bytes = cv.off;
   return L;
 }
 
 template <int D, int RP>
-msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
-                            const KvParams& kp, cudaStream_t st) {
+msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const KvParams& kp,
+                            int grid, cudaStream_t st) {
   using C = KvCfg<D, RP>;
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
   std::call_once(once, [] { attr = set_smem(kvouter_kernel<D, RP>, C::kSmemBytes); });
   if (attr != MSA_OK) return attr;
   ProfScope ps(kPKvOuter, st);
-  kvouter_kernel<D, RP><<<num_sms(), kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, kp);
+  kvouter_kernel<D, RP><<<grid, kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, kp);
   MSA_CHECK_LAUNCH();
   return MSA_OK;
 }
 
 template <int D>
 msa_status_t dispatch_kvouter(int R, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const CUtensorMap& to, const KvParams& kp, cudaStream_t st) {
-  if (R <= 8) return launch_kvouter<D, 8>(tq, tk, tv, to, kp, st);
-  return launch_kvouter<D, 16>(tq, tk, tv, to, kp, st);
+                              const KvParams& kp, int grid, cudaStream_t st) {
+  if (R <= 8) return launch_kvouter<D, 8>(tq, tk, tv, kp, grid, st);
+  return launch_kvouter<D, 16>(tq, tk, tv, kp, grid, st);
 }
 
 // The streaming merge: a ring of shared-memory stages, each holding one (query, group) slab
 // of partials plus its (m, l) pairs and ids; as many stages as fit ~200 KB, 2 at least.
-msa_status_t launch_merge_stream(const MergeParams& mp, int d, cudaStream_t st) {
+msa_status_t launch_merge_stream(const MergeParams& mp, int d, int max_grid, cudaStream_t st) {
   MergeStreamLayout L{};
   const int kR = mp.k * mp.R;
   L.slab_bytes = kR * d * 2;
@@ -537,7 +545,7 @@ msa_status_t launch_merge_stream(const MergeParams& mp, int d, cudaStream_t st) 
   });
   if (attr != MSA_OK) return attr;
   const int64_t units = mp.rows * mp.G;
-  const int grid = int(std::min<int64_t>(num_sms(), units));
+  const int grid = int(std::min<int64_t>(max_grid, units));
   {
     ProfScope ps(kPMerge, st);
     if (d == 128) merge_stream_kernel<128><<<grid, kMergeThreads, smem, st>>>(mp, L);
@@ -557,6 +565,65 @@ msa_status_t set_csr_smem() {
   return attr;
 }
 
+// Chunk overlap. The KV-outer pass of chunk c + 1 (bound by the exp unit and the MMA chain)
+// runs on the caller's stream while the merge of chunk c (bound by HBM) runs on a second
+// stream, each on its own share of the SMs: kvouter launches sms - merge_sms persistent CTAs
+// and the merge merge_sms, so both are resident at once. The partials and (m, l) pairs are
+// double-buffered by chunk parity. The first KV-outer pass and the last merge run alone and
+// take every SM. MSA_MERGE_SMS overrides the merge's share (0 runs the chunks back to back).
+int merge_sm_count(int sms) {
+  static int v = [] {
+    const char* e = std::getenv("MSA_MERGE_SMS");
+    return e ? std::atoi(e) : kDefaultMergeSms;
+  }();
+  return std::max(0, std::min(v, sms / 2));
+}
+
+// The second stream of the calling device (created once per device and kept).
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static cudaStream_t streams[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 0 || dev >= 64) return nullptr;
+  if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+    streams[dev] = nullptr;
+  return streams[dev];
+}
+
+// Events of one call, released when the call returns (the driver frees them once they complete).
+struct EventSet {
+  std::vector<cudaEvent_t> ev;
+  bool make(size_t n) {
+    ev.assign(n, nullptr);
+    for (auto& e : ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    return true;
+  }
+  ~EventSet() {
+    for (auto e : ev)
+      if (e) cudaEventDestroy(e);
+  }
+};
+
+// Joins the side stream back into the caller's stream when a call returns, on success or
+// after an error, so that no merge is still in flight on memory the caller may reuse.
+struct SideJoin {
+  cudaStream_t st = nullptr, side = nullptr;
+  ~SideJoin() {
+    if (side == nullptr) return;
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) {
+      cudaStreamSynchronize(side);
+      return;
+    }
+    cudaEventRecord(e, side);
+    cudaStreamWaitEvent(st, e, 0);
+    cudaEventDestroy(e);
+  }
+};
+
 msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const int32_t* block_ids, int64_t n,
                              int32_t hq, int32_t g, int32_t d, int32_t k, float scale, void* o, void* ws,
                              int64_t query_chunk, cudaStream_t st) {
@@ -568,7 +635,7 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
   AttnLayout L = attn_layout(ws, n, hq, g, d, k, query_chunk);
   const int64_t nb = (n + 127) / 128;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(float(d));
-  CUtensorMap tq, tk, tv, to;
+  CUtensorMap tq, tk, tv;
   const uint64_t panels = uint64_t(d) / 64;
   // q as (64 elems, hq heads, panels, n): one box = 8 heads x all panels of one query
   if ((s = make_map_4d(&tq, q, {64, uint64_t(hq), panels, uint64_t(n)},
@@ -581,16 +648,19 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
   if ((s = make_map_3d(&tv, v, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
-  const int64_t slot_rows = L.chunk_blocks * 128 * g * k;
-  // partials [rows][R][d] as (64 elems, R heads, panels, rows); R >= 8: one box per 8 heads
-  // covering all panels, R < 8: one box per panel
-  if ((s = make_map_4d(&to, L.opart, {64, uint64_t(R), panels, uint64_t(slot_rows)},
-                       {uint64_t(d) * 2, 128, uint64_t(R) * d * 2},
-                       {64, uint32_t(std::min(R, 8)), R >= 8 ? uint32_t(panels) : 1u, 1},
-                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
-    return s;
-  for (int64_t qa0 = 0; qa0 < nb; qa0 += L.chunk_blocks) {
+  const int sms = num_sms();
+  const int msms = L.chunks > 1 ? merge_sm_count(sms) : 0;
+  cudaStream_t side = msms > 0 ? side_stream() : nullptr;
+  const bool overlap = side != nullptr;
+  EventSet kv_done, m_done;   // per chunk: KV-outer pass done (caller's stream), merge done (side stream)
+  if (overlap && (!kv_done.make(size_t(L.chunks)) || !m_done.make(size_t(L.chunks))))
+    return fail(MSA_ERR_CUDA, "cudaEventCreateWithFlags failed");
+  SideJoin join;   // declared after the events: it runs first when the call returns
+  if (overlap) { join.st = st; join.side = side; }
+  int64_t ci = 0;
+  for (int64_t qa0 = 0; qa0 < nb; qa0 += L.chunk_blocks, ++ci) {
     const int64_t qa1 = std::min(nb, qa0 + L.chunk_blocks);
+    const int buf = int(ci & 1);
     CsrParams cp{};
     cp.block_ids = block_ids;
     cp.N = n;
@@ -630,13 +700,24 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     kp.nbk = int(qa1);
     kp.row0 = qa0 * 128;
     kp.scale_log2 = scale * 1.4426950408889634f;
-    kp.ml = L.ml;
-    if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, to, kp, st);
-    else s = dispatch_kvouter<64>(R, tq, tk, tv, to, kp, st);
+    kp.ml = L.ml[buf];
+    kp.opart = static_cast<uint16_t*>(L.opart[buf]);
+    // buffer `buf` was last read by the merge of chunk ci - 2
+    if (overlap && ci >= 2 && cudaStreamWaitEvent(st, m_done.ev[ci - 2], 0) != cudaSuccess)
+      return fail(MSA_ERR_CUDA, "cudaStreamWaitEvent failed");
+    const int kv_grid = (overlap && ci > 0) ? sms - msms : sms;
+    if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, kp, kv_grid, st);
+    else s = dispatch_kvouter<64>(R, tq, tk, tv, kp, kv_grid, st);
     if (s != MSA_OK) return s;
+    cudaStream_t mst = st;
+    if (overlap) {
+      if (cudaEventRecord(kv_done.ev[ci], st) != cudaSuccess || cudaStreamWaitEvent(side, kv_done.ev[ci], 0) != cudaSuccess)
+        return fail(MSA_ERR_CUDA, "cross-stream event failed");
+      mst = side;
+    }
     MergeParams mp{};
-    mp.opart = static_cast<const __nv_bfloat16*>(L.opart);
-    mp.ml = L.ml;
+    mp.opart = static_cast<const __nv_bfloat16*>(L.opart[buf]);
+    mp.ml = L.ml[buf];
     mp.block_ids = block_ids;
     mp.o = static_cast<__nv_bfloat16*>(o);
     mp.row0 = qa0 * 128;
@@ -644,9 +725,12 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     mp.G = g;
     mp.R = R;
     mp.k = k;
-    if ((s = launch_merge_stream(mp, d, st)) != MSA_OK) return s;
+    const int m_grid = (!overlap || ci == L.chunks - 1) ? sms : msms;
+    if ((s = launch_merge_stream(mp, d, m_grid, mst)) != MSA_OK) return s;
+    if (overlap && cudaEventRecord(m_done.ev[ci], side) != cudaSuccess)
+      return fail(MSA_ERR_CUDA, "cudaEventRecord failed");
   }
-  return MSA_OK;
+  return MSA_OK;   // the caller's stream resumes once the last merge is done (SideJoin)
 }
 
 // ------------------------------- decode -------------------------------

@@ -281,4 +281,19 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
                : "memory");
 }
 
+// L2 policy for data written once and read back much later (after many MB of other traffic):
+// evicted first, so that it does not push out operands that are still being reused.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// One 32-byte global store (a whole L2 sector); gptr must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* gptr, const uint32_t* r, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8}, %9;" ::"l"(gptr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "l"(policy)
+               : "memory");
+}
+
 }  // namespace msa
