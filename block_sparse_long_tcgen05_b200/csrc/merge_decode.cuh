@@ -110,24 +110,38 @@ __global__ void __launch_bounds__(256, 2) merge_kernel(const __grid_constant__ M
 
 // ------------------------------------------------------------------------------------
 // Streaming variant of the merge for the prefill chunks. One unit = one (query, group): its
-// k * R * D * 2-byte slab of partials is contiguous, so a producer warp brings it into a
-// ring of shared-memory stages with one bulk copy, and loads the unit's (m, l) pairs and
-// block ids into the same stage with plain loads; the consumer threads combine from shared
-// memory (same arithmetic and slot order as merge_kernel) and write o. Keeping several
-// stages in flight per SM is what lets this pass run at HBM bandwidth.
+// k * R * D * 2-byte slab of partials is contiguous, so a producer warp brings it, with the
+// unit's (m, l) pairs and block ids, into a ring of shared-memory stages by bulk copy.
+// kMergeGroups consumer groups of four warps take units in turn. Per unit each warp first
+// turns the (m, l) pairs of the heads it combines into normalised weights
+// w_s = 2^(m_s - M) / sum_t 2^(m_t - M) l_t (one lane per slot), written next to the slab;
+// then every thread combines one 16-byte chunk of one head row over the valid slots in
+// ascending order. Enough groups and stages stay in flight per SM for the pass to run at
+// HBM bandwidth on a fraction of the SMs.
 // ------------------------------------------------------------------------------------
-constexpr int kMergeGroupThreads = 128;                  // one unit at a time per group
-constexpr int kMergeConsumers = 2 * kMergeGroupThreads;   // two groups on alternate units
-constexpr int kMergeThreads = 32 + kMergeConsumers;
+#ifndef MSA_MERGE_GROUPS
+#define MSA_MERGE_GROUPS 3
+#endif
+constexpr int kMergeGroups = MSA_MERGE_GROUPS;   // consumer groups compiled in (S.groups of them run)
+constexpr int kMergeGroupThreads = 128;
+constexpr int kMergeThreads = 32 + kMergeGroups * kMergeGroupThreads;
 
 struct MergeStreamLayout {
   int slab_bytes;   // k * R * D * 2
   int ml_off;       // offset of the (m, l) pairs inside a stage
   int ids_off;      // offset of the block ids
+  int w_off;        // offset of the weights (k * R floats, written by the consumers)
   int stage_bytes;  // multiple of 128
-  int stages;
+  int stages;       // a multiple of groups: unit n takes stage n % stages and group n % groups, so
+                    // every use of a stage is by the same group, in order (mbarrier parity stays
+                    // within one phase)
+  int groups;       // active consumer groups, 1 .. kMergeGroups
   int bulk_meta;    // (m, l) and ids rows are 16-byte multiples: copy them in bulk too
 };
+
+// bf16 pair (low half first) to two floats: a bf16 is the top half of the float it rounds
+__device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
 template <int D>
 __global__ void __launch_bounds__(kMergeThreads, 1)
@@ -151,7 +165,7 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
   const int64_t grid = gridDim.x;
   const int kR = P.k * P.R;
   if (warp == 0) {
-    // ---- producer: slab by bulk copy, (m, l) and ids by plain loads into the same stage
+    // ---- producer: slab by bulk copy, (m, l) and ids by bulk copy or plain loads
     int n = 0;
     for (int64_t u = blockIdx.x; u < units; u += grid, ++n) {
       const int s = n % S.stages;
@@ -165,7 +179,6 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
       const float2* mlsrc = P.ml + u * kR;
       const int32_t* idsrc = P.block_ids + ((P.row0 + il) * P.G + g) * P.k;
       if (lane == 0) {
-        // slab (and, when 16-byte aligned, the (m, l) pairs and ids) by bulk copy
         mbar_arrive_expect_tx(&full[s], S.slab_bytes + (S.bulk_meta ? kR * 8 + P.k * 4 : 0));
         bulk_load_g2s(st, P.opart + u * static_cast<int64_t>(kR) * D, S.slab_bytes, &full[s]);
         if (S.bulk_meta) {
@@ -188,69 +201,79 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
       }
     }
   } else {
-    // ---- consumers: two groups of four warps take alternate units; within a unit, thread
-    // task (r, c) = head r, 16-byte chunk c of its D-wide row. Every slot's (m, l) and data
-    // are read from shared memory before any is combined (independent loads, one wait).
     const int ct = threadIdx.x - 32;
-    const int grp = ct / kMergeGroupThreads;      // 0 or 1
+    const int grp = ct / kMergeGroupThreads;
     const int gt = ct % kMergeGroupThreads;
-    constexpr int CPR = D / 8;
+    const int gw = gt >> 5;                       // warp within the group
+    constexpr int CPR = D / 8;                    // 16-byte chunks per head row
     const int tasks = P.R * CPR;
     const int Hq = P.G * P.R;
     int n = 0;
     for (int64_t u = blockIdx.x; u < units; u += grid, ++n) {
-      if ((n & 1) != grp) continue;
+      if (n % S.groups != grp) continue;
       const int s = n % S.stages;
       const uint32_t ph = static_cast<uint32_t>(n / S.stages);
       if (!mbar_wait(&full[s], ph & 1, abort_flag, kKidMerge)) break;
-      const uint8_t* st = smem + s * S.stage_bytes;
+      uint8_t* st = smem + s * S.stage_bytes;
       const float2* ml = reinterpret_cast<const float2*>(st + S.ml_off);
       const int32_t* ids = reinterpret_cast<const int32_t*>(st + S.ids_off);
-      int nv = 0;
-#pragma unroll 4
-      for (int x = 0; x < P.k; ++x) nv += (ids[x] >= 0) ? 1 : 0;   // valid ids come first
+      float* wt = reinterpret_cast<float*>(st + S.w_off);
+      // valid ids come first (ascending, -1 padded); k <= 32, one lane per slot
+      const int nv = __popc(__ballot_sync(0xffffffffu, lane < P.k && ids[lane] >= 0));
+      // ---- weights of the heads this warp combines (32 is a multiple of CPR, so each head's
+      // tasks belong to one warp and no other warp reads its weights)
+      for (int t0 = gw * 32; t0 < tasks; t0 += kMergeGroupThreads) {
+        const int r_end = min(P.R, (t0 + 32 + CPR - 1) / CPR);
+        for (int r = t0 / CPR; r < r_end; ++r) {
+          const float2 v = (lane < nv) ? ml[lane * P.R + r] : make_float2(-INFINITY, 0.0f);
+          float M = v.x;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+          const float e = (lane < nv) ? ex2_approx(v.x - M) : 0.0f;
+          float W = e * v.y;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+          if (lane < P.k) wt[lane * P.R + r] = (W > 0.0f) ? __fdividef(e, W) : 0.0f;
+        }
+      }
+      __syncwarp();
+      // ---- combine: thread task (r, c) = head r, 16-byte chunk c of its D-wide row
       const int64_t i = P.row0 + u / P.G;
       const int g = static_cast<int>(u % P.G);
       for (int task = gt; task < tasks; task += kMergeGroupThreads) {
         const int r = task / CPR, c = task % CPR;
+        const uint8_t* src = st + (r * D + c * 8) * 2;
+        const int rstride = P.R * D * 2;          // bytes from one slot's row to the next
         float acc[8];
 #pragma unroll
         for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
-        float W = 0.0f;
-        float M4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // row max over the valid slots
-        for (int sl = 0; sl < nv; ++sl) M4[sl & 3] = fmaxf(M4[sl & 3], ml[sl * P.R + r].x);
-        const float M = fmaxf(fmaxf(M4[0], M4[1]), fmaxf(M4[2], M4[3]));
-        for (int s0 = 0; s0 < nv; s0 += 8) {   // batches of 8 slots, ascending
-          float2 mlv[8];
-          uint4 raw[8];
+        for (int s0 = 0; s0 < nv; s0 += 4) {      // 4 slots' loads in flight, combined in order
+          uint4 raw[4];
+          float w[4];
 #pragma unroll
-          for (int x = 0; x < 8; ++x) {
+          for (int x = 0; x < 4; ++x) {
             const int sl = s0 + x;
-            mlv[x] = (sl < nv) ? ml[sl * P.R + r] : make_float2(-INFINITY, 0.0f);
-            raw[x] = (sl < nv) ? *reinterpret_cast<const uint4*>(st + ((sl * P.R + r) * D + c * 8) * 2)
-                               : make_uint4(0, 0, 0, 0);
+            const bool ok = sl < nv;
+            raw[x] = ok ? *reinterpret_cast<const uint4*>(src + sl * rstride) : make_uint4(0, 0, 0, 0);
+            w[x] = ok ? wt[sl * P.R + r] : 0.0f;
           }
 #pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            if (s0 + x < nv) {
-              const float w = ex2_approx(mlv[x].x - M);
-              W = fmaf(w, mlv[x].y, W);
-              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[x]);
-#pragma unroll
-              for (int t = 0; t < 4; ++t) {
-                const float2 f = __bfloat1622float2(h2[t]);
-                acc[2 * t] = fmaf(w, f.x, acc[2 * t]);
-                acc[2 * t + 1] = fmaf(w, f.y, acc[2 * t + 1]);
-              }
-            }
+          for (int x = 0; x < 4; ++x) {
+            acc[0] = fmaf(w[x], bf16lo(raw[x].x), acc[0]);
+            acc[1] = fmaf(w[x], bf16hi(raw[x].x), acc[1]);
+            acc[2] = fmaf(w[x], bf16lo(raw[x].y), acc[2]);
+            acc[3] = fmaf(w[x], bf16hi(raw[x].y), acc[3]);
+            acc[4] = fmaf(w[x], bf16lo(raw[x].z), acc[4]);
+            acc[5] = fmaf(w[x], bf16hi(raw[x].z), acc[5]);
+            acc[6] = fmaf(w[x], bf16lo(raw[x].w), acc[6]);
+            acc[7] = fmaf(w[x], bf16hi(raw[x].w), acc[7]);
           }
         }
-        const float inv = (W > 0.0f) ? 1.0f / W : 0.0f;
         uint4 out;
-        out.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-        out.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-        out.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-        out.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+        out.x = pack_bf16x2(acc[0], acc[1]);
+        out.y = pack_bf16x2(acc[2], acc[3]);
+        out.z = pack_bf16x2(acc[4], acc[5]);
+        out.w = pack_bf16x2(acc[6], acc[7]);
         reinterpret_cast<uint4*>(P.o + (i * Hq + g * P.R + r) * D)[c] = out;
       }
       __syncwarp();

@@ -525,15 +525,19 @@ msa_status_t dispatch_kvouter(int R, const CUtensorMap& tq, const CUtensorMap& t
 }
 
 // The streaming merge: a ring of shared-memory stages, each holding one (query, group) slab
-// of partials plus its (m, l) pairs and ids; as many stages as fit ~200 KB, 2 at least.
+// of partials plus its (m, l) pairs, ids and weights; as many stages as fit ~210 KB (8 at
+// most), rounded down to a multiple of the consumer groups that run.
 msa_status_t launch_merge_stream(const MergeParams& mp, int d, int max_grid, cudaStream_t st) {
   MergeStreamLayout L{};
   const int kR = mp.k * mp.R;
   L.slab_bytes = kR * d * 2;
   L.ml_off = (L.slab_bytes + 15) / 16 * 16;
   L.ids_off = (L.ml_off + kR * 8 + 15) / 16 * 16;
-  L.stage_bytes = (L.ids_off + mp.k * 4 + 127) / 128 * 128;
-  L.stages = std::max(2, std::min(8, (200 * 1024) / L.stage_bytes));
+  L.w_off = (L.ids_off + mp.k * 4 + 15) / 16 * 16;
+  L.stage_bytes = (L.w_off + kR * 4 + 127) / 128 * 128;
+  const int fit = std::min(8, (210 * 1024) / L.stage_bytes);
+  L.groups = std::max(1, std::min(kMergeGroups, fit));
+  L.stages = std::max(1, fit / L.groups * L.groups);
   L.bulk_meta = (kR % 2 == 0 && mp.k % 4 == 0) ? 1 : 0;
   const int smem = L.stages * L.stage_bytes + L.stages * 16 + 16 + 128;
   if (smem > 227 * 1024) return fail(MSA_ERR_UNSUPPORTED, "merge stage of %d bytes too large", L.stage_bytes);
