@@ -184,7 +184,7 @@ def run_ours(args, world, rank, local):
     cfg = synth.CONFIGS[args.workload]
     inp = synth.prefill_inputs(cfg, device=dev, seed=mdist.rank_seed(cfg.seed, rank))
     N = cfg.N
-    p = msa.prefill_params(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k)
+    p = msa.prefill_params(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k, query_chunk=args.query_chunk)
     ws = torch.empty(msa.msa_forward_workspace(p), dtype=torch.uint8, device=dev)
     o = torch.empty_like(inp["q"])
     ids = torch.empty(N, cfg.G, cfg.k, dtype=torch.int32, device=dev)
@@ -222,7 +222,7 @@ def run_ours(args, world, rank, local):
     dom_launches, dom_ms = stats[dom]
     per_launch_ms = dom_ms / dom_launches
     traffic = args.traffic.get(dom) if args.traffic else None
-    if dom == "index_blockmax":
+    if dom in ("index_blockmax", "index_topk"):
         work = accounting.index_kernel_flops(0, nb, cfg.G, cfg.d_idx) / (dom_launches / args.steps)
         ach = work / (per_launch_ms * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
@@ -329,6 +329,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--query-chunk", type=int, default=0,
+                    help="queries per KV-outer chunk (multiple of 128; 0: the library default, 16384)")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"),
                     help="per-kernel DRAM bytes per launch from an ncu capture (null when absent)")
     args = ap.parse_args()

@@ -31,8 +31,9 @@ def decode_useful_flops(lengths, Hq: int, G: int, d: int, d_idx: int, Bk: int, k
 
 
 def index_kernel_flops(qb_begin: int, qb_end: int, G: int, d_idx: int, Bk: int = 128) -> float:
-    """index_blockmax: every (query, key) pair whose key block lies before the query's
-    own block, i.e. Bk * Bk * qb pairs for query block qb, 2 * d_idx FLOPs each."""
+    """Index Branch score kernels (index_topk, and index_blockmax on the two-kernel path):
+    every (query, key) pair whose key block lies before the query's own block, i.e.
+    Bk * Bk * qb pairs for query block qb, 2 * d_idx FLOPs each."""
     qb = np.arange(qb_begin, qb_end, dtype=np.float64)
     return 2.0 * d_idx * G * Bk * Bk * float(qb.sum())
 
@@ -59,7 +60,7 @@ def main_branch_bytes(N: int, Hq: int, G: int, d: int, Bk: int, k: int) -> dict:
     i = np.arange(N, dtype=np.int64)
     nsel = float(np.minimum(i // Bk + 1, k).sum())       # (query, slot) pairs per group
     R = Hq // G
-    partial = nsel * G * R * (d * 2 + 4)                 # bf16 partial row + fp32 lse
+    partial = nsel * G * R * (d * 2 + 8)                 # bf16 partial row + fp32 (m, l) pair
     q_bytes = N * Hq * d * 2
     kv_bytes = 2 * N * G * d * 2
     return {"kvouter": q_bytes + kv_bytes + partial,

@@ -460,6 +460,20 @@ msa_status_t static_scratch_address(void** out) {
 }
 
 // ------------------------------- main branch (prefill) -------------------------------
+// Chunk overlap. The KV-outer pass of chunk c + 1 (bound by the exp unit and the MMA chain)
+// runs on the caller's stream while the merge of chunk c (bound by HBM) runs on a second
+// stream, each on its own share of the SMs: kvouter launches sms - merge_sms persistent CTAs
+// and the merge merge_sms, so both are resident at once. The partials and (m, l) pairs are
+// double-buffered by chunk parity. The first KV-outer pass and the last merge run alone and
+// take every SM. MSA_MERGE_SMS overrides the merge's share (0 runs the chunks back to back).
+int merge_sm_count(int sms) {
+  static int v = [] {
+    const char* e = std::getenv("MSA_MERGE_SMS");
+    return e ? std::atoi(e) : kDefaultMergeSms;
+  }();
+  return std::max(0, std::min(v, sms / 2));
+}
+
 struct AttnLayout {
   int64_t chunk_blocks = 0;   // query blocks per chunk
   int64_t chunks = 0;
@@ -493,7 +507,7 @@ AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, in
   L.istart = static_cast<uint32_t*>(cv.take(size_t(nbuck + 1) * 4));
   L.entries = static_cast<int32_t*>(cv.take(size_t(max_entries) * 4));
   L.items = static_cast<int4*>(cv.take(size_t(max_items) * 16));
-  const int nbuf = L.chunks > 1 ? 2 : 1;
+  const int nbuf = (L.chunks > 1 && merge_sm_count(num_sms()) > 0) ? 2 : 1;   // overlap needs two
   for (int i = 0; i < nbuf; ++i) {
     L.opart[i] = cv.take(size_t(max_entries) * R * d * 2);
     L.ml[i] = static_cast<float2*>(cv.take(size_t(max_entries) * R * 8));
@@ -569,20 +583,6 @@ msa_status_t set_csr_smem() {
   return attr;
 }
 
-// Chunk overlap. The KV-outer pass of chunk c + 1 (bound by the exp unit and the MMA chain)
-// runs on the caller's stream while the merge of chunk c (bound by HBM) runs on a second
-// stream, each on its own share of the SMs: kvouter launches sms - merge_sms persistent CTAs
-// and the merge merge_sms, so both are resident at once. The partials and (m, l) pairs are
-// double-buffered by chunk parity. The first KV-outer pass and the last merge run alone and
-// take every SM. MSA_MERGE_SMS overrides the merge's share (0 runs the chunks back to back).
-int merge_sm_count(int sms) {
-  static int v = [] {
-    const char* e = std::getenv("MSA_MERGE_SMS");
-    return e ? std::atoi(e) : kDefaultMergeSms;
-  }();
-  return std::max(0, std::min(v, sms / 2));
-}
-
 // The second stream of the calling device (created once per device and kept).
 cudaStream_t side_stream() {
   static std::mutex mu;
@@ -653,7 +653,7 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
   const int sms = num_sms();
-  const int msms = L.chunks > 1 ? merge_sm_count(sms) : 0;
+  const int msms = (L.chunks > 1 && L.opart[1] != L.opart[0]) ? merge_sm_count(sms) : 0;
   cudaStream_t side = msms > 0 ? side_stream() : nullptr;
   const bool overlap = side != nullptr;
   EventSet kv_done, m_done;   // per chunk: KV-outer pass done (caller's stream), merge done (side stream)
