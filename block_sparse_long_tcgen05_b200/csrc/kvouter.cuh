@@ -16,7 +16,7 @@
 //   the unnormalised O (bf16) and (m, l) go to the query's slot s; a later pass merges
 //   the k slots of every query (no atomics).
 //
-// Roles (16 warps):
+// Roles (4 + 4 * kKvSoftmaxWGs + 4 warps; 20 with three softmax warpgroups):
 //   warp 0        TMA loads of K_b and V_b (two buffers each: the next item's block loads
 //                 while the current one is still in use)
 //   warp 1        tcgen05.mma issue of S = Q K^T, in tile order
@@ -24,10 +24,11 @@
 //   warp 3        tcgen05.mma issue of O = P V, in tile order. Two issuers, because an issue
 //                 sequence stalls while the tensor pipe is busy: a PV that is ready does not
 //                 wait behind the S product of the next tile, nor the other way round.
-//   warps 4..7    softmax warpgroup 0 (tiles with even index)
-//   warps 8..11   softmax warpgroup 1 (odd tiles): the two alternate on the exp unit
-//   warps 12..15  epilogue warpgroup: O from TMEM to bf16, stored straight to the partials
-// Tile n uses TMEM pair w = n % 2 (S/P at column 128*w, O at 256 + 128*w).
+//   softmax       kKvSoftmaxWGs warpgroups from warp 4 on; tile n goes to warpgroup
+//                 n % kKvSoftmaxWGs, which takes S(n) from TMEM region n % kKvSoftmaxWGs and
+//                 writes P over it; the warpgroups take turns on the exp unit
+//   epilogue      the last warpgroup: O from TMEM to bf16, stored straight to the partials
+// TMEM: S/P regions at columns 128 * w, w < kKvSoftmaxWGs; O region(s) after them.
 //
 // Shared-memory layouts (all 128-byte swizzled, 1024-byte aligned):
 //   K, V: [panel][128 keys][128 B]                     (8-row group stride 1 KB, panel 16 KB)
@@ -38,8 +39,19 @@
 namespace msa {
 
 constexpr int kKvItemTiles = 8;
-constexpr int kKvThreads = 512;
 constexpr int kKvQStages = 3;
+// Softmax warpgroups = S/P regions of TMEM (128 columns each). Tile n goes to warpgroup
+// n % kKvSoftmaxWGs; with three, a warpgroup's next tile can start its S product while the
+// other two run their softmax, and O (128 columns) is single-buffered: the epilogue hands it
+// back within a few hundred cycles of the PV product.
+#ifndef MSA_KV_SOFTMAX_WGS
+#define MSA_KV_SOFTMAX_WGS 3
+#endif
+constexpr int kKvSoftmaxWGs = MSA_KV_SOFTMAX_WGS;
+constexpr int kKvOBufs = (kKvSoftmaxWGs == 2) ? 2 : 1;
+static_assert(kKvSoftmaxWGs * 128 + kKvOBufs * 128 <= 512, "TMEM holds 512 columns");
+constexpr int kKvEpiWarp = 4 + 4 * kKvSoftmaxWGs;   // first warp of the epilogue warpgroup
+constexpr int kKvThreads = 32 * (kKvEpiWarp + 4);
 
 template <int D, int RP>
 struct KvCfg {
@@ -84,12 +96,14 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* v_empty = bars + 6;             // [2]
   uint64_t* q_full = bars + 8;              // [QS]
   uint64_t* q_empty = bars + 8 + QS;        // [QS]
-  uint64_t* s_full = bars + 8 + 2 * QS;     // [2] S of tile n in TMEM (S issuer -> softmax)
-  uint64_t* p_full = s_full + 2;            // [2] P written over S (softmax, 4 warps -> PV issuer)
-  uint64_t* o_full = s_full + 4;            // [2] PV done (PV issuer -> epilogue; also frees S/P)
-  uint64_t* o_free = s_full + 6;            // [2] O read out (epilogue, 4 warps -> PV issuer)
-  uint64_t* s_done = s_full + 8;            // all S products of the CTA complete
-  uint64_t* pv_done = s_full + 9;           // all PV products of the CTA complete
+  constexpr int NB = kKvSoftmaxWGs, NO = kKvOBufs;
+  uint64_t* s_full = bars + 8 + 2 * QS;     // [NB] S of tile n in TMEM (S issuer -> softmax)
+  uint64_t* p_full = s_full + NB;           // [NB] P written over S (softmax, 4 warps -> PV issuer)
+  uint64_t* sp_free = p_full + NB;          // [NB] PV done: S/P region free (PV issuer -> S issuer)
+  uint64_t* o_full = sp_free + NB;          // [NO] PV done (PV issuer -> epilogue)
+  uint64_t* o_free = o_full + NO;           // [NO] O read out (epilogue, 4 warps -> PV issuer)
+  uint64_t* s_done = o_free + NO;           // all S products of the CTA complete
+  uint64_t* pv_done = s_done + 1;           // all PV products of the CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -101,10 +115,8 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
     }
     for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4);
-      mbar_init(&o_full[i], 1); mbar_init(&o_free[i], 4);
-    }
+    for (int i = 0; i < NB; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4); mbar_init(&sp_free[i], 1); }
+    for (int i = 0; i < NO; ++i) { mbar_init(&o_full[i], 1); mbar_init(&o_free[i], 4); }
     mbar_init(s_done, 1);
     mbar_init(pv_done, 1);
     *abort_flag = 0;
@@ -196,10 +208,10 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------ MMA issuers ------------------------------
-    // warp 1: S(n) once its query rows and its item's K are in shared memory and PV(n - 2),
+    // warp 1: S(n) once its query rows and its item's K are in shared memory and PV(n - NB),
     //         which read P from the same TMEM columns, has completed.
     // warp 3: PV(n) once P(n) is written, its item's V is in shared memory and the epilogue
-    //         has read O(n - 2) out of the same TMEM columns.
+    //         has read O(n - NO) out of the same TMEM columns.
     if (lane == 0) {
       const bool is_s = (warp == 1);
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
@@ -217,12 +229,14 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t v_addr = smem_u32(smem + C::kVOff + kb * C::kTileBytes);
         if (!mbar_wait(is_s ? &k_full[kb] : &v_full[kb], ph, abort_flag, kKidKvOuter)) { ok = false; break; }
         for (int j = 0; j < ntiles; ++j, ++n) {
-          const int w = n & 1;
-          const uint32_t u = static_cast<uint32_t>(n >> 1);
+          const int w = n % NB;                                   // S/P region and warpgroup
+          const uint32_t u = static_cast<uint32_t>(n / NB) & 1;   // phase parity of region w
+          const int ob = n % NO;                                  // O region
+          const uint32_t uo = static_cast<uint32_t>(n / NO) & 1;
           if (is_s) {
             const int qs = n % QS;
             if (!mbar_wait(&q_full[qs], static_cast<uint32_t>(n / QS) & 1, abort_flag, kKidKvOuter) ||
-                !mbar_wait(&o_full[w], (u & 1) ^ 1, abort_flag, kKidKvOuter)) {
+                !mbar_wait(&sp_free[w], u ^ 1, abort_flag, kKidKvOuter)) {
               ok = false;
               break;
             }
@@ -240,19 +254,20 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             umma_commit(&s_full[w]);
             if (j == ntiles - 1) umma_commit(&k_empty[kb]);
           } else {
-            if (!mbar_wait(&p_full[w], u & 1, abort_flag, kKidKvOuter) ||
-                !mbar_wait(&o_free[w], (u & 1) ^ 1, abort_flag, kKidKvOuter)) {
+            if (!mbar_wait(&p_full[w], u, abort_flag, kKidKvOuter) ||
+                !mbar_wait(&o_free[ob], uo ^ 1, abort_flag, kKidKvOuter)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t d_o = tmem + 256 + w * 128;
+            const uint32_t d_o = tmem + NB * 128 + ob * 128;
             const uint32_t a_p = tmem + w * 128;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk)
               umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(v_addr + kk * 2048, 16384, 1024, kLayoutSw128), idesc_o,
                            kk > 0);
-            umma_commit(&o_full[w]);
+            umma_commit(&sp_free[w]);
+            umma_commit(&o_full[ob]);
             if (j == ntiles - 1) umma_commit(&v_empty[kb]);
           }
         }
@@ -262,11 +277,11 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       umma_commit(done);
       mbar_wait(done, 0, nullptr, kKidKvOuter);
     }
-  } else if (warp >= 12) {
+  } else if (warp >= kKvEpiWarp) {
     // ------------------------------ epilogue warpgroup ------------------------------
     // O of every tile: TMEM -> bf16 -> the partial row of (query, slot, head), one 32-byte
-    // store per 16 columns. The TMEM columns are handed back as soon as the last load has
-    // landed; the stores follow from registers.
+    // store per 16 columns, 32 columns at a time. The TMEM columns are handed back as soon
+    // as the last load has landed.
     const int quad = warp & 3;
     const int m = quad * 32 + lane;
     const int q = m / RP, r = m % RP;
@@ -281,35 +296,36 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int g = it.x / P.nbk;
       const int ntiles = (it.z + TQ - 1) / TQ;
       for (int j = 0; j < ntiles; ++j, ++nt) {
-        const int w = nt & 1;
-        const uint32_t u = static_cast<uint32_t>(nt >> 1);
+        const int ob = nt % NO;
+        const uint32_t uo = static_cast<uint32_t>(nt / NO) & 1;
         const int nq = min(TQ, it.z - j * TQ);
         const bool valid = (q < nq) && (r < P.R);
         const int e = valid ? __ldg(P.entries + it.y + j * TQ + q) : 0;
-        const uint32_t t_o = tmem + lane_base + 256 + w * 128;
-        if (!mbar_wait(&o_full[w], u & 1, abort_flag, kKidKvOuter)) { fail = true; break; }
-        tc_fence_after();
-        uint32_t pk[D / 2];
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          uint32_t v[2][32];
-          tmem_ld32(t_o + c * 64, v[0]);
-          tmem_ld32(t_o + c * 64 + 32, v[1]);
-          tmem_ld_wait();
-          if (c == D / 64 - 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&o_free[w]);
-          }
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            pk[c * 32 + x] = pack_bf16x2(__uint_as_float(v[x >> 4][(2 * x) & 31]), __uint_as_float(v[x >> 4][(2 * x + 1) & 31]));
-        }
+        uint16_t* dst = P.opart;
         if (valid) {
           const int64_t il = static_cast<int64_t>(e >> 5) - P.row0;
-          uint16_t* dst = P.opart + (((il * P.G + g) * P.k + (e & 31)) * P.R + r) * D;
+          dst += (((il * P.G + g) * P.k + (e & 31)) * P.R + r) * D;
+        }
+        const uint32_t t_o = tmem + lane_base + NB * 128 + ob * 128;
+        if (!mbar_wait(&o_full[ob], uo, abort_flag, kKidKvOuter)) { fail = true; break; }
+        tc_fence_after();
 #pragma unroll
-          for (int z = 0; z < D / 16; ++z) st_global_v8(dst + z * 16, pk + z * 8, policy);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_o + c * 32, v);
+          tmem_ld_wait();
+          if (c == D / 32 - 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_free[ob]);
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1]));
+          if (valid) {
+            st_global_v8(dst + c * 32, pk, policy);
+            st_global_v8(dst + c * 32 + 16, pk + 8, policy);
+          }
         }
       }
     }
@@ -317,7 +333,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------ softmax warpgroups ------------------------------
     // The four warps of a warpgroup never wait for one another: each hands its rows over
     // through mbarrier arrivals (P to the PV issuer).
-    const int wg = (warp - 4) >> 2;               // 0 or 1: takes tiles with nt % 2 == wg
+    const int wg = (warp - 4) >> 2;               // takes tiles with nt % NB == wg
     const int quad = warp & 3;
     const int m = quad * 32 + lane;               // row of the tile == TMEM lane
     const int q = m / RP, r = m % RP;
@@ -332,8 +348,8 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int g = it.x / P.nbk, b = it.x % P.nbk;
       const int ntiles = (it.z + TQ - 1) / TQ;
       for (int j = 0; j < ntiles; ++j, ++nt) {
-        if ((nt & 1) != wg) continue;
-        const uint32_t u = static_cast<uint32_t>(nt >> 1);
+        if (nt % NB != wg) continue;
+        const uint32_t u = static_cast<uint32_t>(nt / NB);
         const int nq = min(TQ, it.z - j * TQ);
         const bool valid = (q < nq) && (r < P.R);
         const int e = (pref_nt == nt) ? e_pref : (valid ? __ldg(P.entries + it.y + j * TQ + q) : 0);
@@ -342,14 +358,14 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // load the entry for this warpgroup's next tile now (same item or the next one); rows
         // past that tile's queries read a neighbouring entry that is never used
         {
-          int jn = j + 2;
+          int jn = j + NB;
           const int32_t* base = nullptr;
           if (jn < ntiles) {
             base = P.entries + it.y;
           } else if (t + grid < n_items && (jn -= ntiles) < (nxt.z + TQ - 1) / TQ) {
             base = P.entries + nxt.y;
           }
-          pref_nt = base ? nt + 2 : -1;
+          pref_nt = base ? nt + NB : -1;
           if (base) e_pref = __ldg(base + jn * TQ + q);
         }
         const int limit = !valid ? -1 : ((b == (i >> 7)) ? (i & 127) : 127);   // keys c <= limit are visible
