@@ -34,11 +34,25 @@ SPEC_BF16_TFLOPS = 2250.0
 FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-def source_sha256() -> str:
+# Device sources each kernel is built from: DRAM counters taken on a kernel describe it only
+# while these files are unchanged.
+KERNEL_SOURCES = {
+    "index_topk": ["index_topk.cuh", "index_blockmax.cuh", "topk.cuh", "ptx.cuh", "common.cuh"],
+    "index_blockmax": ["index_blockmax.cuh", "ptx.cuh", "common.cuh"],
+    "topk_prefill": ["topk.cuh", "ptx.cuh", "common.cuh"],
+    "kvouter": ["kvouter.cuh", "ptx.cuh", "common.cuh"],
+    "merge": ["merge_decode.cuh", "ptx.cuh", "common.cuh"],
+}
+
+
+def kernel_sha256(kernel: str, csrc: str | None = None) -> str | None:
     import hashlib
+    files = KERNEL_SOURCES.get(kernel)
+    if files is None:
+        return None
+    csrc = csrc or os.path.join(ROOT, "block_sparse_long_tcgen05_b200", "csrc")
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "block_sparse_long_tcgen05_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in files:
         h.update(f.encode())
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()
@@ -337,9 +351,11 @@ def main():
     args.traffic = {}
     if args.traffic_json and os.path.exists(args.traffic_json):
         tj = json.load(open(args.traffic_json))
-        # counters only describe the kernels they were taken on: drop them once the source changed
-        if tj.get("source_sha256") == source_sha256():
-            args.traffic = tj.get(args.workload, {})
+        # counters only describe the kernels they were taken on: drop a kernel's figure once
+        # its device source changed
+        for kern, ent in tj.get(args.workload, {}).items():
+            if isinstance(ent, dict) and ent.get("source_sha256") == kernel_sha256(kern):
+                args.traffic[kern] = ent["bytes"]
     world, rank, local = dist_setup()
     try:
         if args.impl == "reference":

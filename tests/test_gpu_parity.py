@@ -48,19 +48,35 @@ def check_prefill(cfg, rows=None, query_chunk=0, check_all_ids=True):
     msa.check_device_error()
     if rows is None:
         rows = list(range(cfg.N))
-    ids_ref, o_ref = orc.prefill_rows(inp, rows, cfg.Bk, cfg.k)
+    if cfg.N * cfg.Hq * cfg.d > (1 << 31):
+        # long sequences: the oracle reads the device tensors row by row (one group's index
+        # keys at a time) instead of taking a host copy of every input
+        ids_ref, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, cfg.Bk, cfg.k)
+        o_ref = orc.attend_rows(inp["q"], inp["k"], inp["v"], ids_ref, rows, cfg.Bk)
+    else:
+        ids_ref, o_ref = orc.prefill_rows(inp, rows, cfg.Bk, cfg.k)
     ids_g = ids_gpu.cpu().numpy()
     np.testing.assert_array_equal(ids_g[rows], ids_ref)
     if check_all_ids:
-        # structural rules on every row: count, ascending, local block present
-        i = np.arange(cfg.N)
-        bl = i // cfg.Bk
-        valid = ids_g >= 0
-        assert np.array_equal(valid.sum(-1), np.broadcast_to(np.minimum(cfg.k, bl + 1)[:, None], valid.shape[:2]))
-        last = np.take_along_axis(ids_g, (valid.sum(-1, keepdims=True) - 1), axis=-1)[..., 0]
-        assert np.array_equal(last, np.broadcast_to(bl[:, None], last.shape))
-    assert_close(o.float().cpu().numpy()[rows], o_ref, "prefill o")
+        structural_ids_check(ids_g, cfg.Bk, cfg.k)
+    rt = torch.as_tensor(rows, device=o.device)
+    assert_close(o[rt].float().cpu().numpy(), o_ref, "prefill o")
     return inp, ids_gpu, o
+
+
+def structural_ids_check(ids_g, Bk, k):
+    """Rules every row must satisfy: min(k, bl + 1) valid ids, ascending, -1 padded, the
+    local block last."""
+    N = ids_g.shape[0]
+    bl = np.arange(N) // Bk
+    valid = ids_g >= 0
+    nval = valid.sum(-1)
+    assert np.array_equal(nval, np.broadcast_to(np.minimum(k, bl + 1)[:, None], nval.shape))
+    assert not np.any(valid[..., 1:] & ~valid[..., :-1])          # -1 padding only at the end
+    both = valid[..., 1:] & valid[..., :-1]
+    assert np.all(np.diff(ids_g, axis=-1)[both] > 0)                  # strictly ascending
+    last = np.take_along_axis(ids_g, (nval[..., None] - 1), axis=-1)[..., 0]
+    assert np.array_equal(last, np.broadcast_to(bl[:, None], last.shape))
 
 
 # ---------------------------------------------------------------- Index Branch alone
@@ -157,6 +173,14 @@ def test_forward_32k_sampled(cuda_ok):
 def test_forward_128k_sampled(cuda_ok):
     """The headline 128K configuration, in the launch configuration the bench times."""
     check_prefill(synth.P128K, rows=sample_rows(131072, 16, n=48, seed=2), check_all_ids=True)
+
+
+@pytest.mark.slow
+def test_forward_1m_sampled(cuda_ok):
+    """The 1M-token configuration: the two-kernel Index Branch (block maxima in chunks of at
+    most 4 GiB) and 64 query chunks of the Main Branch; sampled rows against the oracle,
+    structural rules on every row."""
+    check_prefill(synth.P1M, rows=sample_rows(1 << 20, 16, n=10, seed=3), check_all_ids=True)
 
 
 # ---------------------------------------------------------------- decode
