@@ -41,7 +41,7 @@ KERNEL_SOURCES = {
     "index_blockmax": ["index_blockmax.cuh", "ptx.cuh", "common.cuh"],
     "topk_prefill": ["topk.cuh", "ptx.cuh", "common.cuh"],
     "kvouter": ["kvouter.cuh", "ptx.cuh", "common.cuh"],
-    "merge": ["merge_decode.cuh", "ptx.cuh", "common.cuh"],
+    "merge": ["merge.cuh", "ptx.cuh", "common.cuh"],
 }
 
 

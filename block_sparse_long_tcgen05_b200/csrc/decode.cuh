@@ -1,0 +1,238 @@
+// Query-stationary decode kernels: Index Branch scan of one new query per sequence and the
+// sparse attention over its selected blocks (merged by merge_kernel).
+#pragma once
+#include <cuda_bf16.h>
+
+#include "merge.cuh"
+#include "ptx.cuh"
+
+namespace msa {
+
+// ------------------------------------------------------------------------------------
+// Decode, Index Branch: block maxima of the one new query per sequence against every
+// full block before its local block (query-stationary: the index-key cache streams
+// through once, 64 contiguous bytes per lane per load).
+// ------------------------------------------------------------------------------------
+struct DecodeScanParams {
+  const __nv_bfloat16* q_idx;   // [B][G][DI]
+  const __nv_bfloat16* k_idx;   // [B][Lmax][G][DI]
+  const int32_t* seqlens;
+  uint32_t* maxima;             // [B][G][nbmax]
+  int B, G, nbmax;
+  int64_t Lmax;
+};
+
+// grid (nbmax, B), 256 threads: one CTA per (sequence, block). Needs G * DI / 32 to be
+// a power of two <= 32 (checked by the host).
+template <int DI>
+__global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant__ DecodeScanParams P) {
+  __shared__ uint32_t smax[32];
+  const int b = blockIdx.y, kb = blockIdx.x;
+  const int L = P.seqlens[b];
+  if (L < 1 || L > P.Lmax) {
+    if (kb == 0 && threadIdx.x == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidDecodeScan);
+    return;
+  }
+  const int bl = (L - 1) / 128;
+  if (kb >= bl) return;
+  const int cpt = P.G * DI / 32;             // 64-byte chunks per token
+  constexpr int LPG = DI / 32;               // lanes (chunks) per group
+  const int lane = threadIdx.x & 31;
+  const int w = lane % cpt;                  // constant per lane since cpt | 32
+  const int g = w / LPG;
+  const int qoff = (w % LPG) * 32;
+  if (threadIdx.x < 32) smax[threadIdx.x] = 0u;
+  float qv[32];
+  {
+    const uint4* qp = reinterpret_cast<const uint4*>(P.q_idx + (static_cast<int64_t>(b) * P.G + g) * DI + qoff);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint4 raw = __ldg(qp + u);
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const float2 f = __bfloat1622float2(h2[t]);
+        qv[u * 8 + 2 * t] = f.x;
+        qv[u * 8 + 2 * t + 1] = f.y;
+      }
+    }
+  }
+  __syncthreads();
+  const uint4* base = reinterpret_cast<const uint4*>(P.k_idx + (static_cast<int64_t>(b) * P.Lmax + kb * 128) *
+                                                                   P.G * DI);
+  const int nchunks = 128 * cpt;
+  float best = -INFINITY;
+  for (int c0 = threadIdx.x; c0 < nchunks; c0 += 256 * 2) {
+    uint4 raw[2][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int c = c0 + h * 256;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) raw[h][u] = (c < nchunks) ? __ldg(base + static_cast<int64_t>(c) * 4 + u) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float acc = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[h][u]);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float2 f = __bfloat1622float2(h2[t]);
+          acc = fmaf(qv[u * 8 + 2 * t], f.x, acc);
+          acc = fmaf(qv[u * 8 + 2 * t + 1], f.y, acc);
+        }
+      }
+#pragma unroll
+      for (int o = 1; o < LPG; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (c0 + h * 256 < nchunks) best = fmaxf(best, acc);
+    }
+  }
+  if ((lane % LPG) == 0) {
+    float m = __fadd_rn(best, 0.0f);
+    uint32_t u = __float_as_uint(m);
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    atomicMax(&smax[g], u);
+  }
+  __syncthreads();
+  if (threadIdx.x < P.G) P.maxima[(static_cast<int64_t>(b) * P.G + threadIdx.x) * P.nbmax + kb] = smax[threadIdx.x];
+}
+
+// ------------------------------------------------------------------------------------
+// Decode, Main Branch: one CTA per (sequence, group, slot): exact softmax attention of
+// the group's R heads over the slot's block (causal in the local block), written as an
+// unnormalised partial with its (row max, row sum) for the merge kernel.
+// ------------------------------------------------------------------------------------
+// 16-byte asynchronous global -> shared copy (bypassing L1); with ok == false nothing is
+// read and the 16 shared bytes are zero-filled. Both addresses 16-byte aligned.
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, bool ok) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(sdst)), "l"(gsrc), "r"(ok ? 16 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+struct DecodeAttnParams {
+  const __nv_bfloat16* q;       // [B][Hq][D]
+  const __nv_bfloat16* kc;      // [B][Lmax][G][D]
+  const __nv_bfloat16* vc;
+  const int32_t* seqlens;
+  const int32_t* block_ids;     // [B][G][k]
+  __nv_bfloat16* opart;         // [B][G][k][R][D]
+  float2* ml;                   // [B][G][k][R]
+  int B, G, R, k;
+  int64_t Lmax;
+  float scale_log2;
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant__ DecodeAttnParams P) {
+  constexpr int KS = D + 8;    // padded smem row (bank spread)
+  extern __shared__ uint8_t dsm[];
+  __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(dsm);
+  __nv_bfloat16* Vs = Ks + 128 * KS;
+  float* Qs = reinterpret_cast<float*>(Vs + 128 * KS);   // [R][D]
+  float* Ss = Qs + P.R * D;                              // [R][128]
+  float* stat = Ss + P.R * 128;                          // [R][2]: max, 1/sum
+  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int blk = P.block_ids[(static_cast<int64_t>(b) * P.G + g) * P.k + s];
+  if (blk < 0) return;
+  const int L = P.seqlens[b];
+  const int pos = L - 1;
+  if (L < 1 || L > P.Lmax || blk > pos / 128) {
+    if (threadIdx.x == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidDecodeAttn);
+    return;
+  }
+  const int j0 = blk * 128;
+  const int nvalid = min(128, pos - j0 + 1);
+  const int tid = threadIdx.x;
+  // q rows, pre-scaled into log2 units
+  for (int e = tid; e < P.R * D; e += 128) {
+    const int r = e / D, dd = e % D;
+    Qs[e] = __bfloat162float(P.q[(static_cast<int64_t>(b) * P.G * P.R + g * P.R + r) * D + dd]) * P.scale_log2;
+  }
+  // K / V rows of the block, 16-byte asynchronous copies all in flight at once (rows past
+  // the query are zero-filled: source size 0)
+  constexpr int CPR = D / 8;
+  for (int e = tid; e < 128 * CPR; e += 128) {
+    const int j = e / CPR, c = e % CPR;
+    const bool ok = j < nvalid;
+    const int64_t off = ok ? ((static_cast<int64_t>(b) * P.Lmax + j0 + j) * P.G + g) * D + c * 8 : 0;
+    cp_async16(Ks + j * KS + c * 8, P.kc + off, ok);
+    cp_async16(Vs + j * KS + c * 8, P.vc + off, ok);
+  }
+  cp_async_wait_all();
+  __syncthreads();
+  // scores: thread = key
+  {
+    const int j = tid;
+    for (int r = 0; r < P.R; ++r) {
+      float acc = 0.0f;
+      if (j < nvalid) {
+#pragma unroll 4
+        for (int c = 0; c < CPR; ++c) {
+          const uint4 raw = *reinterpret_cast<const uint4*>(Ks + j * KS + c * 8);
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const float2 f = __bfloat1622float2(h2[t]);
+            acc = fmaf(Qs[r * D + c * 8 + 2 * t], f.x, acc);
+            acc = fmaf(Qs[r * D + c * 8 + 2 * t + 1], f.y, acc);
+          }
+        }
+      }
+      Ss[r * 128 + j] = (j < nvalid) ? acc : -INFINITY;
+    }
+  }
+  __syncthreads();
+  // softmax per head: warp w takes heads w, w + 4, ...
+  {
+    const int w = tid >> 5, lane = tid & 31;
+    for (int r = w; r < P.R; r += 4) {
+      float v4[4];
+      float mx = -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { v4[u] = Ss[r * 128 + lane + 32 * u]; mx = fmaxf(mx, v4[u]); }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float sum = 0.0f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { v4[u] = exp2f(v4[u] - mx); sum += v4[u]; Ss[r * 128 + lane + 32 * u] = v4[u]; }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+      if (lane == 0) { stat[2 * r] = mx; stat[2 * r + 1] = sum; }
+    }
+  }
+  __syncthreads();
+  const int64_t slot = (static_cast<int64_t>(b) * P.G + g) * P.k + s;
+  // O = P V: task (r, c) = head r, 8 columns c*8 .. c*8 + 7; 16-byte V loads, keys in order
+  for (int e = tid; e < P.R * CPR; e += 128) {
+    const int r = e / CPR, c = e % CPR;
+    float acc[8];
+#pragma unroll
+    for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
+#pragma unroll 4
+    for (int j = 0; j < nvalid; ++j) {
+      const float w = Ss[r * 128 + j];
+      const uint4 raw = *reinterpret_cast<const uint4*>(Vs + j * KS + c * 8);
+      acc[0] = fmaf(w, bf16lo(raw.x), acc[0]);
+      acc[1] = fmaf(w, bf16hi(raw.x), acc[1]);
+      acc[2] = fmaf(w, bf16lo(raw.y), acc[2]);
+      acc[3] = fmaf(w, bf16hi(raw.y), acc[3]);
+      acc[4] = fmaf(w, bf16lo(raw.z), acc[4]);
+      acc[5] = fmaf(w, bf16hi(raw.z), acc[5]);
+      acc[6] = fmaf(w, bf16lo(raw.w), acc[6]);
+      acc[7] = fmaf(w, bf16hi(raw.w), acc[7]);
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(P.opart + (slot * P.R + r) * D + c * 8) = out;
+  }
+  if (tid < P.R) P.ml[slot * P.R + tid] = make_float2(stat[2 * tid], stat[2 * tid + 1]);
+}
+
+}  // namespace msa

@@ -18,7 +18,8 @@
 #include "index_blockmax.cuh"
 #include "index_topk.cuh"
 #include "kvouter.cuh"
-#include "merge_decode.cuh"
+#include "merge.cuh"
+#include "decode.cuh"
 #include "topk.cuh"
 
 using namespace msa;
