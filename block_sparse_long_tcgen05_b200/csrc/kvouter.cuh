@@ -16,7 +16,7 @@
 //   the unnormalised O (bf16) and (m, l) go to the query's slot s; a later pass merges
 //   the k slots of every query (no atomics).
 //
-// Roles (4 + 4 * kKvSoftmaxWGs + 4 warps; 20 with three softmax warpgroups):
+// Roles (4 + 4 * kKvSoftmaxWGs + 4 warps; 16 with two softmax warpgroups):
 //   warp 0        TMA loads of K_b and V_b (two buffers each: the next item's block loads
 //                 while the current one is still in use)
 //   warp 1        tcgen05.mma issue of S = Q K^T, in tile order
@@ -27,25 +27,26 @@
 //   softmax       kKvSoftmaxWGs warpgroups from warp 4 on; tile n goes to warpgroup
 //                 n % kKvSoftmaxWGs, which takes S(n) from TMEM region n % kKvSoftmaxWGs and
 //                 writes P over it; the warpgroups take turns on the exp unit
-//   epilogue      the last warpgroup: O from TMEM to bf16, stored straight to the partials
+//   epilogue      the last warpgroup: O from TMEM to bf16 staging, TMA-stored per query
 // TMEM: S/P regions at columns 128 * w, w < kKvSoftmaxWGs; O region(s) after them.
 //
 // Shared-memory layouts (all 128-byte swizzled, 1024-byte aligned):
 //   K, V: [panel][128 keys][128 B]                     (8-row group stride 1 KB, panel 16 KB)
-//   Q: [8-row group][panel][8 rows][128 B]             (8-row group stride kPanels KB, panel 1 KB)
+//   Q, O staging: [8-row group][panel][8 rows][128 B]  (8-row group stride kPanels KB, panel 1 KB)
 #pragma once
 #include "ptx.cuh"
 
 namespace msa {
 
 constexpr int kKvItemTiles = 8;
-constexpr int kKvQStages = 3;
+constexpr int kKvQStages = 2;
 // Softmax warpgroups = S/P regions of TMEM (128 columns each). Tile n goes to warpgroup
-// n % kKvSoftmaxWGs; with three, a warpgroup's next tile can start its S product while the
-// other two run their softmax, and O (128 columns) is single-buffered: the epilogue hands it
-// back within a few hundred cycles of the PV product.
+// n % kKvSoftmaxWGs. Two (the default): O is double-buffered and every thread may hold 128
+// registers. Three: a warpgroup's next tile can start its S product while the other two run
+// their softmax, O (128 columns) is single-buffered, and the 640 threads get 96 registers
+// each (measured slower at d = 128: the softmax then spills).
 #ifndef MSA_KV_SOFTMAX_WGS
-#define MSA_KV_SOFTMAX_WGS 3
+#define MSA_KV_SOFTMAX_WGS 2
 #endif
 constexpr int kKvSoftmaxWGs = MSA_KV_SOFTMAX_WGS;
 constexpr int kKvOBufs = (kKvSoftmaxWGs == 2) ? 2 : 1;
@@ -62,7 +63,8 @@ struct KvCfg {
   static constexpr int kKOff = 0;                        // 2 K buffers
   static constexpr int kVOff = 2 * kTileBytes;           // 2 V buffers
   static constexpr int kQOff = 4 * kTileBytes;           // kKvQStages query stages
-  static constexpr int kBarOff = kQOff + kKvQStages * kTileBytes;
+  static constexpr int kStgOff = kQOff + kKvQStages * kTileBytes;   // O staging (one tile)
+  static constexpr int kBarOff = kStgOff + kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
@@ -74,16 +76,18 @@ struct KvParams {
   int64_t row0;              // first query of the chunk
   float scale_log2;
   float2* ml;                // [chunk rows][G][k][R]: (row max in log2 units, row sum)
-  uint16_t* opart;           // [chunk rows][G][k][R][D] bf16: unnormalised partial outputs
 };
 
 // tensor maps:
 //   tm_q: 4-D view of q [N][Hq][D] as (64 elems, Hq heads, D/64 panels, N), box (64, 8, D/64, 1)
 //   tm_k, tm_v: 3-D view of k / v [N][G][D] as (D, G, N), box (64, 1, 128)
+//   tm_o: 4-D view of the partials [rows][R][D] as (64, R, D/64, rows),
+//         box (64, min(R, 8), R >= 8 ? D/64 : 1, 1)
 template <int D, int RP>
 __global__ void __launch_bounds__(kKvThreads, 1)
 kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ KvParams P) {
+               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+               const __grid_constant__ KvParams P) {
   using C = KvCfg<D, RP>;
   constexpr int TQ = C::TQ;
   constexpr int QS = kKvQStages;
@@ -279,14 +283,16 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp >= kKvEpiWarp) {
     // ------------------------------ epilogue warpgroup ------------------------------
-    // O of every tile: TMEM -> bf16 -> the partial row of (query, slot, head), one 32-byte
-    // store per 16 columns, 32 columns at a time. The TMEM columns are handed back as soon
-    // as the last load has landed.
+    // O of every tile: TMEM -> bf16 -> this warp's 32 rows of the swizzled staging tile; then
+    // lane q of the warp issues the TMA stores of the warp's q-th query (2 KB: all its heads),
+    // so each partial row leaves as whole lines. A warp reuses its staging rows once its own
+    // stores have read them; the TMEM columns are handed back as soon as the last load lands.
     const int quad = warp & 3;
     const int m = quad * 32 + lane;
-    const int q = m / RP, r = m % RP;
+    constexpr int QPW = 32 / RP;                  // queries whose rows this warp holds
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
-    const uint64_t policy = l2_policy_evict_first();
+    const uint32_t o_row = smem_u32(smem + C::kStgOff) + (m >> 3) * C::kGroupBytes + (m & 7) * 128;
+    if (lane == 0) tma_prefetch_desc(&tm_o);
     int nt = 0;
     bool fail = false;
     int4 nxt = first_item;
@@ -299,16 +305,14 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int ob = nt % NO;
         const uint32_t uo = static_cast<uint32_t>(nt / NO) & 1;
         const int nq = min(TQ, it.z - j * TQ);
-        const bool valid = (q < nq) && (r < P.R);
-        const int e = valid ? __ldg(P.entries + it.y + j * TQ + q) : 0;
-        uint16_t* dst = P.opart;
-        if (valid) {
-          const int64_t il = static_cast<int64_t>(e >> 5) - P.row0;
-          dst += (((il * P.G + g) * P.k + (e & 31)) * P.R + r) * D;
-        }
+        const int qw = quad * QPW + lane;         // the query whose stores this lane issues
+        const bool st_lane = (lane < QPW) && (qw < nq);
+        const int e = st_lane ? __ldg(P.entries + it.y + j * TQ + qw) : 0;
         const uint32_t t_o = tmem + lane_base + NB * 128 + ob * 128;
         if (!mbar_wait(&o_full[ob], uo, abort_flag, kKidKvOuter)) { fail = true; break; }
         tc_fence_after();
+        if (lane < QPW) bulk_wait_read_all();     // previous tile's stores have read the rows
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t v[32];
@@ -319,16 +323,35 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_free[ob]);
           }
-          uint32_t pk[16];
 #pragma unroll
-          for (int x = 0; x < 16; ++x) pk[x] = pack_bf16x2(__uint_as_float(v[2 * x]), __uint_as_float(v[2 * x + 1]));
-          if (valid) {
-            st_global_v8(dst + c * 32, pk, policy);
-            st_global_v8(dst + c * 32 + 16, pk + 8, policy);
+          for (int x = 0; x < 4; ++x) {              // four 16-byte chunks of 8 columns
+            const int ch = c * 4 + x;                // chunk index along d
+            const uint32_t* s8 = v + x * 8;
+            st_shared_v4(o_row + (ch >> 3) * 1024 + (((ch & 7) ^ (m & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(s8[0]), __uint_as_float(s8[1])),
+                         pack_bf16x2(__uint_as_float(s8[2]), __uint_as_float(s8[3])),
+                         pack_bf16x2(__uint_as_float(s8[4]), __uint_as_float(s8[5])),
+                         pack_bf16x2(__uint_as_float(s8[6]), __uint_as_float(s8[7])));
           }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (st_lane) {
+          const int64_t il = static_cast<int64_t>(e >> 5) - P.row0;
+          const int row = static_cast<int>((il * P.G + g) * P.k + (e & 31));
+          const uint8_t* src = smem + C::kStgOff + qw * (RP / 8) * C::kGroupBytes;
+          if (P.R >= 8) {
+#pragma unroll
+            for (int h8 = 0; h8 < RP / 8; ++h8) tma_store_4d(&tm_o, src + h8 * C::kGroupBytes, 0, h8 * 8, 0, row);
+          } else {
+#pragma unroll
+            for (int p = 0; p < C::kPanels; ++p) tma_store_4d(&tm_o, src + p * 1024, 0, 0, p, row);
+          }
+          bulk_commit_group();
         }
       }
     }
+    if (lane < QPW) bulk_wait_all();              // every store of this lane has completed
   } else if (warp >= 4) {
     // ------------------------------ softmax warpgroups ------------------------------
     // The four warps of a warpgroup never wait for one another: each hands its rows over

@@ -519,24 +519,24 @@ AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, in
 }
 
 template <int D, int RP>
-msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const KvParams& kp,
-                            int grid, cudaStream_t st) {
+msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
+                            const KvParams& kp, int grid, cudaStream_t st) {
   using C = KvCfg<D, RP>;
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
   std::call_once(once, [] { attr = set_smem(kvouter_kernel<D, RP>, C::kSmemBytes); });
   if (attr != MSA_OK) return attr;
   ProfScope ps(kPKvOuter, st);
-  kvouter_kernel<D, RP><<<grid, kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, kp);
+  kvouter_kernel<D, RP><<<grid, kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, kp);
   MSA_CHECK_LAUNCH();
   return MSA_OK;
 }
 
 template <int D>
 msa_status_t dispatch_kvouter(int R, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                              const KvParams& kp, int grid, cudaStream_t st) {
-  if (R <= 8) return launch_kvouter<D, 8>(tq, tk, tv, kp, grid, st);
-  return launch_kvouter<D, 16>(tq, tk, tv, kp, grid, st);
+                              const CUtensorMap& to, const KvParams& kp, int grid, cudaStream_t st) {
+  if (R <= 8) return launch_kvouter<D, 8>(tq, tk, tv, to, kp, grid, st);
+  return launch_kvouter<D, 16>(tq, tk, tv, to, kp, grid, st);
 }
 
 // The streaming merge: a ring of shared-memory stages, each holding one (query, group) slab
@@ -640,7 +640,7 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
   AttnLayout L = attn_layout(ws, n, hq, g, d, k, query_chunk);
   const int64_t nb = (n + 127) / 128;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(float(d));
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to[2];
   const uint64_t panels = uint64_t(d) / 64;
   // q as (64 elems, hq heads, panels, n): one box = 8 heads x all panels of one query
   if ((s = make_map_4d(&tq, q, {64, uint64_t(hq), panels, uint64_t(n)},
@@ -653,6 +653,15 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
   if ((s = make_map_3d(&tv, v, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
+  const int64_t slot_rows = L.chunk_blocks * 128 * g * k;
+  // partials [rows][R][d] as (64 elems, R heads, panels, rows); R >= 8: one box per 8 heads
+  // covering all panels, R < 8: one box per panel
+  for (int i = 0; i < 2; ++i)
+    if ((s = make_map_4d(&to[i], L.opart[i], {64, uint64_t(R), panels, uint64_t(slot_rows)},
+                         {uint64_t(d) * 2, 128, uint64_t(R) * d * 2},
+                         {64, uint32_t(std::min(R, 8)), R >= 8 ? uint32_t(panels) : 1u, 1},
+                         CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+      return s;
   const int sms = num_sms();
   const int msms = (L.chunks > 1 && L.opart[1] != L.opart[0]) ? merge_sm_count(sms) : 0;
   cudaStream_t side = msms > 0 ? side_stream() : nullptr;
@@ -706,13 +715,12 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     kp.row0 = qa0 * 128;
     kp.scale_log2 = scale * 1.4426950408889634f;
     kp.ml = L.ml[buf];
-    kp.opart = static_cast<uint16_t*>(L.opart[buf]);
     // buffer `buf` was last read by the merge of chunk ci - 2
     if (overlap && ci >= 2 && cudaStreamWaitEvent(st, m_done.ev[ci - 2], 0) != cudaSuccess)
       return fail(MSA_ERR_CUDA, "cudaStreamWaitEvent failed");
     const int kv_grid = (overlap && ci > 0) ? sms - msms : sms;
-    if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, kp, kv_grid, st);
-    else s = dispatch_kvouter<64>(R, tq, tk, tv, kp, kv_grid, st);
+    if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, to[buf], kp, kv_grid, st);
+    else s = dispatch_kvouter<64>(R, tq, tk, tv, to[buf], kp, kv_grid, st);
     if (s != MSA_OK) return s;
     cudaStream_t mst = st;
     if (overlap) {
