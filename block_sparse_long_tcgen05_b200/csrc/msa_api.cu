@@ -584,18 +584,21 @@ msa_status_t set_csr_smem() {
   return attr;
 }
 
-// The second stream of the calling device (created once per device and kept).
-cudaStream_t side_stream() {
+// Extra streams of the calling device, created once per device and kept: kind 0 runs the
+// overlapped merges, kind 1 the host-to-device copies and kind 2 the device-to-host copies of
+// msa_forward_host.
+cudaStream_t aux_stream(int kind) {
   static std::mutex mu;
-  static cudaStream_t streams[64] = {};
+  static cudaStream_t streams[3][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   std::lock_guard<std::mutex> lk(mu);
-  if (dev < 0 || dev >= 64) return nullptr;
-  if (streams[dev] == nullptr && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-    streams[dev] = nullptr;
-  return streams[dev];
+  if (dev < 0 || dev >= 64 || kind < 0 || kind > 2) return nullptr;
+  cudaStream_t& s = streams[kind][dev];
+  if (s == nullptr && cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) s = nullptr;
+  return s;
 }
+cudaStream_t side_stream() { return aux_stream(0); }
 
 // Events of one call, released when the call returns (the driver frees them once they complete).
 struct EventSet {
@@ -629,9 +632,13 @@ struct SideJoin {
   }
 };
 
+// chunk_in (optional, one event per chunk): the caller's stream waits for chunk_in[c] before
+// chunk c's kernels (its query rows and the key/value rows up to its end must be resident).
+// chunk_out (optional): recorded after chunk c's merge, once o's rows of chunk c are final.
 msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const int32_t* block_ids, int64_t n,
                              int32_t hq, int32_t g, int32_t d, int32_t k, float scale, void* o, void* ws,
-                             int64_t query_chunk, cudaStream_t st) {
+                             int64_t query_chunk, cudaStream_t st, const cudaEvent_t* chunk_in = nullptr,
+                             const cudaEvent_t* chunk_out = nullptr) {
   msa_status_t s;
   if ((s = set_csr_smem()) != MSA_OK) return s;
   const int R = hq / g;
@@ -675,6 +682,8 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
   for (int64_t qa0 = 0; qa0 < nb; qa0 += L.chunk_blocks, ++ci) {
     const int64_t qa1 = std::min(nb, qa0 + L.chunk_blocks);
     const int buf = int(ci & 1);
+    if (chunk_in && cudaStreamWaitEvent(st, chunk_in[ci], 0) != cudaSuccess)
+      return fail(MSA_ERR_CUDA, "cudaStreamWaitEvent failed");
     CsrParams cp{};
     cp.block_ids = block_ids;
     cp.N = n;
@@ -741,6 +750,8 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     const int m_grid = (!overlap || ci == L.chunks - 1) ? sms : msms;
     if ((s = launch_merge_stream(mp, d, m_grid, mst)) != MSA_OK) return s;
     if (overlap && cudaEventRecord(m_done.ev[ci], side) != cudaSuccess)
+      return fail(MSA_ERR_CUDA, "cudaEventRecord failed");
+    if (chunk_out && cudaEventRecord(chunk_out[ci], mst) != cudaSuccess)
       return fail(MSA_ERR_CUDA, "cudaEventRecord failed");
   }
   return MSA_OK;   // the caller's stream resumes once the last merge is done (SideJoin)
@@ -1038,6 +1049,114 @@ msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, cons
     return run_decode(p, q, k, v, q_idx, k_idx, block_ids_out, o, workspace, st);
   }
   return fail(MSA_ERR_INVALID_ARG, "mode=%d", p->mode);
+}
+
+// Device buffer of msa_forward_host: device copies of the five inputs and of o, then the
+// msa_forward workspace (whose first bytes hold the block ids).
+struct HostLayout {
+  void *q, *k, *v, *qi, *ki, *o, *ws;
+  size_t ws_bytes, bytes;
+};
+static HostLayout host_layout(void* base, const msa_params* p) {
+  Carver cv(base);
+  HostLayout H{};
+  const size_t n = size_t(p->n);
+  H.q = cv.take(n * p->hq * p->d * 2);
+  H.k = cv.take(n * p->g * p->d * 2);
+  H.v = cv.take(n * p->g * p->d * 2);
+  H.qi = cv.take(n * p->g * p->d_idx * 2);
+  H.ki = cv.take(n * p->g * p->d_idx * 2);
+  H.o = cv.take(n * p->hq * p->d * 2);
+  H.ws_bytes = msa_forward_workspace(p);
+  H.ws = cv.take(H.ws_bytes);
+  H.bytes = cv.off;
+  return H;
+}
+
+size_t msa_forward_host_device_bytes(const msa_params* p) {
+  if (!p || p->mode != MSA_MODE_PREFILL || msa_forward_workspace(p) == 0) return 0;
+  return host_layout(nullptr, p).bytes;
+}
+
+msa_status_t msa_forward_host(const msa_params* p, const void* q, const void* k, const void* v, const void* q_idx,
+                              const void* k_idx, int32_t* block_ids_out, void* o, void* device_buf,
+                              size_t device_bytes, void* stream) {
+  g_detail[0] = 0;
+  if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->mode != MSA_MODE_PREFILL) return fail(MSA_ERR_UNSUPPORTED, "msa_forward_host takes prefill only");
+  msa_status_t s;
+  if ((s = check_common(p->n, p->g, p->bk, p->k)) != MSA_OK) return s;
+  if ((s = check_main_dims(p->hq, p->g, p->d)) != MSA_OK) return s;
+  if ((s = check_d_idx(p->d_idx)) != MSA_OK) return s;
+  if (!(p->scale >= 0.0f) || std::isinf(p->scale)) return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (p->query_chunk < 0 || p->query_chunk % 128 != 0)
+    return fail(MSA_ERR_INVALID_ARG, "query_chunk=%lld must be a non-negative multiple of 128", (long long)p->query_chunk);
+  if ((s = check_ptr(q, "q")) != MSA_OK || (s = check_ptr(k, "k")) != MSA_OK || (s = check_ptr(v, "v")) != MSA_OK ||
+      (s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
+      (s = check_ptr(o, "o")) != MSA_OK || (s = check_ptr(device_buf, "device_buf")) != MSA_OK)
+    return s;
+  if (block_ids_out && (s = check_ptr(block_ids_out, "block_ids_out")) != MSA_OK) return s;
+  const size_t need = msa_forward_host_device_bytes(p);
+  if (device_bytes < need) return fail(MSA_ERR_WORKSPACE, "device buffer %zu bytes < %zu needed", device_bytes, need);
+  const HostLayout H = host_layout(device_buf, p);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaStream_t cin = aux_stream(1), cout = aux_stream(2);
+  if (cin == nullptr || cout == nullptr) return fail(MSA_ERR_CUDA, "could not create the copy streams");
+  const int64_t n = p->n;
+  const AttnLayout L = attn_layout(nullptr, n, p->hq, p->g, p->d, p->k, p->query_chunk);
+  const int64_t rows_per_chunk = L.chunk_blocks * 128;
+  EventSet ev;   // 0 start, 1 index inputs in, 2 selection done, then per chunk: rows in, rows out
+  if (!ev.make(size_t(3 + 2 * L.chunks))) return fail(MSA_ERR_CUDA, "cudaEventCreateWithFlags failed");
+  const cudaEvent_t* chunk_in = ev.ev.data() + 3;
+  const cudaEvent_t* chunk_out = ev.ev.data() + 3 + L.chunks;
+  SideJoin join_in, join_out;   // whatever happens, `stream` waits for both copy streams
+  join_in.st = st; join_in.side = cin;
+  join_out.st = st; join_out.side = cout;
+  auto cuda_ok = [](cudaError_t e) { return e == cudaSuccess; };
+  // the device buffer may still be in use by earlier work on `stream`
+  if (!cuda_ok(cudaEventRecord(ev.ev[0], st)) || !cuda_ok(cudaStreamWaitEvent(cin, ev.ev[0], 0)) ||
+      !cuda_ok(cudaStreamWaitEvent(cout, ev.ev[0], 0)))
+    return fail(MSA_ERR_CUDA, "stream ordering failed");
+  // index inputs first, alone on the link, so the Index Branch starts as early as possible
+  const size_t idx_bytes = size_t(n) * p->g * p->d_idx * 2;
+  if (!cuda_ok(cudaMemcpyAsync(H.qi, q_idx, idx_bytes, cudaMemcpyHostToDevice, st)) ||
+      !cuda_ok(cudaMemcpyAsync(H.ki, k_idx, idx_bytes, cudaMemcpyHostToDevice, st)) ||
+      !cuda_ok(cudaEventRecord(ev.ev[1], st)) || !cuda_ok(cudaStreamWaitEvent(cin, ev.ev[1], 0)))
+    return fail(MSA_ERR_CUDA, "index input copy failed");
+  // then the rows of q, k and v chunk by chunk, behind the Index Branch
+  const size_t qrow = size_t(p->hq) * p->d * 2, krow = size_t(p->g) * p->d * 2;
+  for (int64_t c = 0; c < L.chunks; ++c) {
+    const int64_t r0 = c * rows_per_chunk, r1 = std::min(n, r0 + rows_per_chunk);
+    const size_t nr = size_t(r1 - r0);
+    if (!cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(H.q) + r0 * qrow, static_cast<const uint8_t*>(q) + r0 * qrow,
+                                 nr * qrow, cudaMemcpyHostToDevice, cin)) ||
+        !cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(H.k) + r0 * krow, static_cast<const uint8_t*>(k) + r0 * krow,
+                                 nr * krow, cudaMemcpyHostToDevice, cin)) ||
+        !cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(H.v) + r0 * krow, static_cast<const uint8_t*>(v) + r0 * krow,
+                                 nr * krow, cudaMemcpyHostToDevice, cin)) ||
+        !cuda_ok(cudaEventRecord(chunk_in[c], cin)))
+      return fail(MSA_ERR_CUDA, "input copy failed");
+  }
+  int32_t* ids = reinterpret_cast<int32_t*>(H.ws);
+  void* rest = static_cast<uint8_t*>(H.ws) + prefill_ids_bytes(n, p->g, p->k);
+  if ((s = run_index_select(H.qi, H.ki, n, p->g, p->d_idx, p->k, ids, rest, st)) != MSA_OK) return s;
+  if (block_ids_out) {
+    if (!cuda_ok(cudaEventRecord(ev.ev[2], st)) || !cuda_ok(cudaStreamWaitEvent(cout, ev.ev[2], 0)) ||
+        !cuda_ok(cudaMemcpyAsync(block_ids_out, ids, size_t(n) * p->g * p->k * 4, cudaMemcpyDeviceToHost, cout)))
+      return fail(MSA_ERR_CUDA, "block id copy failed");
+  }
+  if ((s = run_sparse_attn(H.q, H.k, H.v, ids, n, p->hq, p->g, p->d, p->k, p->scale, H.o, rest, p->query_chunk, st,
+                           chunk_in, chunk_out)) != MSA_OK)
+    return s;
+  // each chunk's output rows go back as soon as its merge is done
+  for (int64_t c = 0; c < L.chunks; ++c) {
+    const int64_t r0 = c * rows_per_chunk, r1 = std::min(n, r0 + rows_per_chunk);
+    if (!cuda_ok(cudaStreamWaitEvent(cout, chunk_out[c], 0)) ||
+        !cuda_ok(cudaMemcpyAsync(static_cast<uint8_t*>(o) + r0 * qrow, static_cast<const uint8_t*>(H.o) + r0 * qrow,
+                                 size_t(r1 - r0) * qrow, cudaMemcpyDeviceToHost, cout)))
+      return fail(MSA_ERR_CUDA, "output copy failed");
+  }
+  return MSA_OK;   // `stream` resumes once both copy streams are done (SideJoin)
 }
 
 msa_status_t msa_profile_start(void) {

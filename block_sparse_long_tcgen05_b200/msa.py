@@ -22,7 +22,8 @@ MODE_PREFILL, MODE_DECODE = 0, 1
 # Every symbol include/msa.h declares.
 EXPORTS = ("msa_index_select_workspace", "msa_index_select", "msa_sparse_attn_workspace", "msa_sparse_attn",
            "msa_forward_workspace", "msa_forward", "msa_get_device_error", "msa_status_string",
-           "msa_last_error_detail", "msa_profile_start", "msa_profile_stop", "msa_index_select_static")
+           "msa_last_error_detail", "msa_profile_start", "msa_profile_stop", "msa_index_select_static",
+           "msa_forward_host_device_bytes", "msa_forward_host")
 
 
 class MsaError(RuntimeError):
@@ -69,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_profile_start": (c_i32, []),
         "msa_profile_stop": (c_i32, [ctypes.POINTER(MsaKernelStat), c_i32]),
         "msa_index_select_static": (c_i32, [c_p, c_p, c_i64, c_i32, c_i32, c_i32, c_i32, c_p, c_p]),
+        "msa_forward_host_device_bytes": (c_sz, [pp]),
+        "msa_forward_host": (c_i32, [pp, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -184,6 +187,38 @@ def msa_forward(p: MsaParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     _check(lib.msa_forward(ctypes.byref(p), _bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(q_idx, "q_idx"),
                            _bf16(k_idx, "k_idx"), _ptr(block_ids), _ptr(o), _ptr(ws), ws.numel(),
                            _stream(q.device)))
+    return o
+
+
+def _host(t: torch.Tensor | None, name: str, dtype=torch.bfloat16) -> int | None:
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} host tensor")
+    return t.data_ptr()
+
+
+def msa_forward_host_device_bytes(p: MsaParams) -> int:
+    return load_library().msa_forward_host_device_bytes(ctypes.byref(p))
+
+
+def forward_host(p: MsaParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, q_idx: torch.Tensor,
+                 k_idx: torch.Tensor, o: torch.Tensor, block_ids: torch.Tensor | None = None,
+                 device_buf: torch.Tensor | None = None, device=None) -> torch.Tensor:
+    """Prefill with host tensors in and out (page-locked for the copies to overlap the
+    kernels); see msa_forward_host in include/msa.h. Enqueued on the current stream of
+    `device`: o (and block_ids) are complete once that stream is."""
+    lib = load_library()
+    device = torch.device("cuda") if device is None else torch.device(device)
+    need = lib.msa_forward_host_device_bytes(ctypes.byref(p))
+    if need == 0:
+        raise MsaError(1, "unsupported or invalid msa_params for msa_forward_host")
+    buf = _workspace(need, device, device_buf)
+    _check(lib.msa_forward_host(ctypes.byref(p), _host(q, "q"), _host(k, "k"), _host(v, "v"), _host(q_idx, "q_idx"),
+                                _host(k_idx, "k_idx"), _host(block_ids, "block_ids", torch.int32), _host(o, "o"),
+                                _ptr(buf), buf.numel() * buf.element_size(), _stream(device)))
     return o
 
 

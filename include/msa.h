@@ -136,6 +136,23 @@ MSA_API msa_status_t msa_forward(const msa_params* p, const void* q, const void*
                          const void* k_idx, int32_t* block_ids_out, void* o, void* workspace,
                          size_t workspace_bytes, void* stream);
 
+/* Prefill with the inputs and the output in HOST memory. q, k, v, q_idx, k_idx and o are
+ * host pointers with the shapes of msa_forward's prefill (block_ids_out: host [n, g, k] or
+ * NULL); page-locked memory lets the copies overlap the kernels (pageable memory works, the
+ * copies then serialise with the host). device_buf (device, 256-byte aligned,
+ * msa_forward_host_device_bytes(p) bytes) receives device copies of the inputs and of o,
+ * and the msa_forward workspace. Within the call the index inputs are copied first, the
+ * Index Branch starts as soon as they land while q / k / v are copied behind it chunk by
+ * chunk (query_chunk rows) on a second stream; each chunk's Main Branch starts once its rows
+ * are resident, and its output rows are copied back on a third stream while later chunks
+ * compute. Everything is ordered after earlier work on `stream`, and the host output (and
+ * block ids) are complete once `stream` is. Prefill only (decode returns
+ * MSA_ERR_UNSUPPORTED). Calls that share `stream` may reuse one device_buf. */
+MSA_API size_t msa_forward_host_device_bytes(const msa_params* p);
+MSA_API msa_status_t msa_forward_host(const msa_params* p, const void* q, const void* k, const void* v,
+                                      const void* q_idx, const void* k_idx, int32_t* block_ids_out, void* o,
+                                      void* device_buf, size_t device_bytes, void* stream);
+
 /* Synchronises `stream`, then reads and clears this device's error word. Returns
  * MSA_OK, MSA_ERR_TIMEOUT or MSA_ERR_DEVICE_BOUNDS (the first error recorded since the
  * last call), or MSA_ERR_CUDA when the synchronisation itself failed. */

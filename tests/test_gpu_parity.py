@@ -183,6 +183,30 @@ def test_forward_1m_sampled(cuda_ok):
     check_prefill(synth.P1M, rows=sample_rows(1 << 20, 16, n=10, seed=3), check_all_ids=True)
 
 
+def test_forward_host_matches_device_path(cuda_ok):
+    """msa_forward_host (host tensors in and out, copies pipelined with the chunks) gives the
+    device path's output and block ids bit for bit; several query chunks and a ragged tail."""
+    cfg = cfg_of(5000, 16, 2, 128, 64, 8, hot=0.1, seed=21)
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    p = msa.prefill_params(cfg.N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k, query_chunk=1024)
+    ids_d = torch.empty(cfg.N, cfg.G, cfg.k, dtype=torch.int32, device="cuda")
+    o_d = msa.msa_forward(p, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], block_ids=ids_d)
+    host = {n: t.cpu().pin_memory() for n, t in inp.items()}
+    o_h = torch.empty(o_d.shape, dtype=o_d.dtype, pin_memory=True)
+    ids_h = torch.empty(ids_d.shape, dtype=torch.int32, pin_memory=True)
+    for _ in range(2):   # the device buffer is reused by the second call
+        o_h.zero_()
+        msa.forward_host(p, host["q"], host["k"], host["v"], host["q_idx"], host["k_idx"], o_h, block_ids=ids_h)
+        torch.cuda.synchronize()
+        msa.check_device_error()
+        assert torch.equal(ids_h, ids_d.cpu())
+        assert torch.equal(o_h, o_d.cpu())
+    rows = sample_rows(cfg.N, cfg.k, n=24, seed=5)
+    ids_ref, o_ref = orc.prefill_rows(inp, rows, cfg.Bk, cfg.k)
+    np.testing.assert_array_equal(ids_h.numpy()[rows], ids_ref)
+    assert_close(o_h.float().numpy()[rows], o_ref, "forward_host o")
+
+
 # ---------------------------------------------------------------- decode
 
 def check_decode(cfg, lengths, seqs=None, Lmax=None):
