@@ -206,9 +206,12 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const IdxTopkItem it = idx_topk_item(P, t);
       const int qb = it.qa + tile;
       const bool tile_present = (tile == 0) || it.has_b;
-      uint64_t L[KM];
+      // running top list: ordered scores (descending) and their block ids; 0 is below every
+      // real ordered score
+      uint32_t Ls[KM];
+      int Lb[KM];
 #pragma unroll
-      for (int p = 0; p < KM; ++p) L[p] = 0ull;   // below every real key (ordered keys are > 0)
+      for (int p = 0; p < KM; ++p) { Ls[p] = 0u; Lb[p] = -1; }
       for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
         const int ab = static_cast<int>(ik & 1);
         const uint32_t au = static_cast<uint32_t>(ik >> 1);
@@ -237,7 +240,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           m = __fadd_rn(m, 0.0f);   // -0 -> +0 so equal scores give equal keys
           uint32_t u = __float_as_uint(m);
           u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-          topk_insert<KM>(L, (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(0xFFFFFFFFu - kb));
+          topk_insert_ascending<KM>(Ls, Lb, u, kb);
         } else {
           tc_fence_before();
           __syncwarp();
@@ -253,7 +256,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       } else {
         int ids[KM];
 #pragma unroll
-        for (int p = 0; p < KM; ++p) ids[p] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(L[p]));
+        for (int p = 0; p < KM; ++p) ids[p] = Lb[p];
 #pragma unroll
         for (int pass = 0; pass < KM; ++pass) {
 #pragma unroll

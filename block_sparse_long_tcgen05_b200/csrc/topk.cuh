@@ -25,6 +25,28 @@ __device__ __forceinline__ void topk_insert(uint64_t (&L)[KM], uint64_t key) {
   }
 }
 
+// The same insertion for a caller that offers the blocks in ascending order of kb: 32-bit
+// ordered scores with the ids alongside. A block never displaces an equal score already in
+// the list (strict comparisons), which is the tie rule (equal scores: the lower block id
+// ranks first), because every block already in the list has a lower id.
+template <int KM>
+__device__ __forceinline__ void topk_insert_ascending(uint32_t (&Ls)[KM], int (&Lb)[KM], uint32_t u, int kb) {
+  static_assert(KM >= 1, "at least one non-local place");
+  if (u > Ls[KM - 1]) {
+#pragma unroll
+    for (int p = KM - 1; p > 0; --p) {
+      const bool down = u > Ls[p - 1];   // the entry above moves down into place p
+      const bool here = u > Ls[p];
+      Ls[p] = down ? Ls[p - 1] : (here ? u : Ls[p]);
+      Lb[p] = down ? Lb[p - 1] : (here ? kb : Lb[p]);
+    }
+    if (u > Ls[0]) {
+      Ls[0] = u;
+      Lb[0] = kb;
+    }
+  }
+}
+
 // Select for one row: src[kb * stride] holds the ordered key of block kb for
 // kb in [0, bl); bl is the local block. Writes KM + 1 ids (ascending) to out.
 // Requires bl >= KM + 1 (more non-local candidates than places).
