@@ -5,13 +5,15 @@
 One step = one msa_forward prefill over the 131072-token sequence (Index Branch: scores +
 block max + Top-k; Main Branch: CSR build + KV-outer attention + LSE merge), inputs
 resident in HBM. Under torchrun every rank runs its own independent sequence (weak
-scaling, no data-path collective); the time is the max over ranks. Rank 0 prints one
-JSON line. `--impl reference` times the fp64 CPU oracle on a bounded sample of query
+scaling), or with --shard groups its range of GQA groups of one shared sequence (strong
+scaling); no data-path collective either way, the time is the max over ranks. Rank 0
+prints one JSON line. `--impl reference` times the fp64 CPU oracle on a bounded sample of query
 rows of the same workload instead (rank 0 only).
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -196,12 +198,26 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     peaks, peak_src = load_peaks()
     cfg = synth.CONFIGS[args.workload]
-    inp = synth.prefill_inputs(cfg, device=dev, seed=mdist.rank_seed(cfg.seed, rank))
+    if args.shard == "groups":
+        # one sequence for the whole job; this rank computes its contiguous range of groups
+        full = synth.prefill_inputs(cfg, device=dev, seed=cfg.seed)
+        inp = mdist.shard_inputs_by_group(full, cfg.G, world, rank)
+        del full
+        torch.cuda.empty_cache()
+        groups, _, _ = mdist.group_slice(cfg.G, cfg.R, world, rank)
+        rcfg = dataclasses.replace(cfg, Hq=len(groups) * cfg.R, G=len(groups))
+        seqs_per_job = 1
+        parallelism = f"GQA groups sharded over {world} GPU(s), one sequence, no collective"
+    else:
+        inp = synth.prefill_inputs(cfg, device=dev, seed=mdist.rank_seed(cfg.seed, rank))
+        rcfg = cfg
+        seqs_per_job = world
+        parallelism = "one independent sequence per GPU, no collective"
     N = cfg.N
-    p = msa.prefill_params(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k, query_chunk=args.query_chunk)
+    p = msa.prefill_params(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.d_idx, rcfg.k, query_chunk=args.query_chunk)
     ws = torch.empty(msa.msa_forward_workspace(p), dtype=torch.uint8, device=dev)
     o = torch.empty_like(inp["q"])
-    ids = torch.empty(N, cfg.G, cfg.k, dtype=torch.int32, device=dev)
+    ids = torch.empty(N, rcfg.G, rcfg.k, dtype=torch.int32, device=dev)
 
     def step():
         msa.msa_forward(p, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], o=o, block_ids=ids,
@@ -220,9 +236,9 @@ def run_ours(args, world, rank, local):
     ms = max_over_ranks(ms, world)
     barrier(world)
 
-    idx_f, main_f = accounting.prefill_useful_flops(N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.Bk, cfg.k)
+    idx_f, main_f = accounting.prefill_useful_flops(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.d_idx, rcfg.Bk, rcfg.k)
     useful_tflops = (idx_f + main_f) / (ms * 1e-3) / 1e12
-    value = world * N / (ms * 1e-3)
+    value = seqs_per_job * N / (ms * 1e-3)   # tokens of the whole job over the slowest rank's time
 
     # per-kernel breakdown (this rank, same timed region)
     stages = {}
@@ -237,20 +253,20 @@ def run_ours(args, world, rank, local):
     per_launch_ms = dom_ms / dom_launches
     traffic = args.traffic.get(dom) if args.traffic else None
     if dom in ("index_blockmax", "index_topk"):
-        work = accounting.index_kernel_flops(0, nb, cfg.G, cfg.d_idx) / (dom_launches / args.steps)
+        work = accounting.index_kernel_flops(0, nb, rcfg.G, rcfg.d_idx) / (dom_launches / args.steps)
         ach = work / (per_launch_ms * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
                 "work_per_launch": work}
     elif dom == "kvouter":
-        work = accounting.kvouter_flops(N, cfg.Hq, cfg.d, cfg.Bk, cfg.k) / (dom_launches / args.steps)
+        work = accounting.kvouter_flops(N, rcfg.Hq, rcfg.d, rcfg.Bk, rcfg.k) / (dom_launches / args.steps)
         ach = work / (per_launch_ms * 1e-3) / 1e12
         roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
                 "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
                 "peak_source": f"{peak_src} bf16 sustained", "work_per_launch": work}
     else:
-        byts = accounting.main_branch_bytes(N, cfg.Hq, cfg.G, cfg.d, cfg.Bk, cfg.k).get(dom, float("nan"))
+        byts = accounting.main_branch_bytes(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.Bk, rcfg.k).get(dom, float("nan"))
         work = byts / (dom_launches / args.steps)
         ach = work / (per_launch_ms * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -258,9 +274,10 @@ def run_ours(args, world, rank, local):
                 "work_per_launch": work}
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if args.shard == "groups" else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
-            "config": workload_config(cfg),
+            "config": workload_config(cfg, {"parallelism": parallelism}),
             "prefill": {"tokens_per_s": value, "useful_tflops": useful_tflops * world,
                         "useful_tflops_per_gpu": useful_tflops,
                         "frac_spec_bf16_2250": useful_tflops / SPEC_BF16_TFLOPS,
@@ -323,7 +340,7 @@ def run_ours(args, world, rank, local):
         barrier(world)
         esteps = max(2, min(args.steps, 10))
         ems = max_over_ranks(timed(estep, esteps, stream), world)
-        line["e2e"] = {"value": world * N / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        line["e2e"] = {"value": seqs_per_job * N / (ems * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": esteps,
                        "api": "msa_forward_host", "output_equals_device_path": same}
         del dbuf, host, o_h
@@ -350,6 +367,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", choices=["sequences", "groups"], default="sequences",
+                    help="N > 1: one independent sequence per GPU (weak scaling) or the GQA groups of one "
+                         "sequence split over the GPUs (strong scaling); no collective either way")
     ap.add_argument("--query-chunk", type=int, default=0,
                     help="queries per KV-outer chunk (multiple of 128; 0: the library default, 16384)")
     ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"),

@@ -1,10 +1,12 @@
 """Multi-GPU plumbing for running the MSA hot path data-parallel.
 
-The path shards without any exchange: each rank owns whole independent sequences (prefill)
-or whole sequences of a decode batch, so the data path has no collective. The only
-cross-rank traffic is timing: a barrier around timed regions and the max of the per-rank
-times (a job is as fast as its slowest rank). One process per GPU; torchrun sets RANK,
-LOCAL_RANK and WORLD_SIZE.
+The path shards without any exchange, two ways: each rank owns whole independent sequences
+(prefill) or whole sequences of a decode batch; or every rank works on the same sequence
+and owns a contiguous range of GQA groups with their query heads (groups never interact:
+each has its own index head and its own block selection, zhichai.net section 2). Either
+way the data path has no collective. The only cross-rank traffic is timing: a barrier
+around timed regions and the max of the per-rank times (a job is as fast as its slowest
+rank). One process per GPU; torchrun sets RANK, LOCAL_RANK and WORLD_SIZE.
 """
 from __future__ import annotations
 
@@ -43,6 +45,24 @@ def shard(n_units: int, world: int, rank: int) -> range:
     base, extra = divmod(n_units, world)
     lo = rank * base + min(rank, extra)
     return range(lo, lo + base + (1 if rank < extra else 0))
+
+
+def group_slice(G: int, R: int, world: int, rank: int) -> tuple[range, slice, slice]:
+    """Group sharding of one sequence: (groups, query-head slice, group slice) of `rank`.
+    Query head h belongs to group h // R, so a contiguous range of groups owns a contiguous
+    range of heads; requires world <= G."""
+    if world > G:
+        raise ValueError(f"{world} ranks for {G} groups")
+    groups = shard(G, world, rank)
+    return groups, slice(groups.start * R, groups.stop * R), slice(groups.start, groups.stop)
+
+
+def shard_inputs_by_group(inp: dict, G: int, world: int, rank: int) -> dict:
+    """This rank's contiguous copies of a prefill input dict (q [N,Hq,d]; k, v, q_idx,
+    k_idx [N,G,*]) for its groups."""
+    R = inp["q"].shape[1] // G
+    _, hs, gs = group_slice(G, R, world, rank)
+    return {n: (t[:, hs] if n == "q" else t[:, gs]).contiguous() for n, t in inp.items()}
 
 
 def max_over_ranks(x: float, device=None) -> float:

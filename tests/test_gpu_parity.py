@@ -207,6 +207,26 @@ def test_forward_host_matches_device_path(cuda_ok):
     assert_close(o_h.float().numpy()[rows], o_ref, "forward_host o")
 
 
+def test_group_shard_equals_slice_of_full_forward(cuda_ok):
+    """Group sharding (bench.py --shard groups): the forward on one rank's groups gives, bit for
+    bit, those groups' heads and block ids of the full forward (two ranks emulated on one GPU,
+    one after the other; no rank waits on another)."""
+    from block_sparse_long_tcgen05_b200 import dist as mdist
+    cfg = cfg_of(3000, 16, 4, 128, 64, 6, hot=0.1, seed=31)
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    ids_full = torch.empty(cfg.N, cfg.G, cfg.k, dtype=torch.int32, device="cuda")
+    o_full = msa.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cfg.k, block_ids=ids_full)
+    world = 2
+    for r in range(world):
+        part = mdist.shard_inputs_by_group(inp, cfg.G, world, r)
+        groups, hs, gs = mdist.group_slice(cfg.G, cfg.R, world, r)
+        ids_p = torch.empty(cfg.N, len(groups), cfg.k, dtype=torch.int32, device="cuda")
+        o_p = msa.prefill(part["q"], part["k"], part["v"], part["q_idx"], part["k_idx"], cfg.k, block_ids=ids_p)
+        msa.check_device_error()
+        assert torch.equal(ids_p, ids_full[:, gs])
+        assert torch.equal(o_p, o_full[:, hs])
+
+
 # ---------------------------------------------------------------- decode
 
 def check_decode(cfg, lengths, seqs=None, Lmax=None):
