@@ -87,6 +87,26 @@ def test_forward_param_validation(lib):
     assert lib.msa_forward(ctypes.byref(d), P, P, P, P, P, None, P, P, 1 << 40, None) == 1   # seqlens NULL
 
 
+def test_forward_host_validation_without_cuda(lib):
+    """msa_forward_host checks everything before it touches a stream: prefill only, pointers,
+    chunking, and the size of the device buffer (inputs + output + the forward workspace)."""
+    P = 1 << 12
+    p = msa.prefill_params(1000, 8, 2, 64, 32, 4)
+    need = lib.msa_forward_host_device_bytes(ctypes.byref(p))
+    io = 1000 * 8 * 64 * 2 * 2 + 2 * 1000 * 2 * 64 * 2 + 2 * 1000 * 2 * 32 * 2   # q, o, k, v, q_idx, k_idx
+    assert need >= io + lib.msa_forward_workspace(ctypes.byref(p))
+    assert lib.msa_forward_host(ctypes.byref(p), P, P, P, P, P, None, P, P, need - 1, None) == 3
+    assert lib.msa_forward_host(ctypes.byref(p), P, None, P, P, P, None, P, P, need, None) == 1
+    assert lib.msa_forward_host(ctypes.byref(p), P, P, P, P, P, None, P + 8, P, need, None) == 1   # unaligned o
+    p.query_chunk = 100
+    assert lib.msa_forward_host_device_bytes(ctypes.byref(p)) == 0
+    assert lib.msa_forward_host(ctypes.byref(p), P, P, P, P, P, None, P, P, 1 << 40, None) == 1
+    d = msa.MsaParams(mode=1, hq=64, g=8, d=128, d_idx=128, bk=128, k=16, scale=0.0, n=4, lmax=1000,
+                      seqlens=None, query_chunk=0)
+    assert lib.msa_forward_host_device_bytes(ctypes.byref(d)) == 0
+    assert lib.msa_forward_host(ctypes.byref(d), P, P, P, P, P, None, P, P, 1 << 40, None) == 2   # decode
+
+
 def test_workspace_sizes_grow_with_problem(lib):
     a = lib.msa_sparse_attn_workspace(32768, 64, 8, 128, 128, 16)
     b = lib.msa_sparse_attn_workspace(131072, 64, 8, 128, 128, 16)
