@@ -5,6 +5,7 @@
 
 #include "merge.cuh"
 #include "ptx.cuh"
+#include "topk.cuh"
 
 namespace msa {
 
@@ -103,6 +104,76 @@ __global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant_
 // the group's R heads over the slot's block (causal in the local block), written as an
 // unnormalised partial with its (row max, row sum) for the merge kernel.
 // ------------------------------------------------------------------------------------
+// Decode Top-k over the scanned block maxima [B][G][nbmax].
+// One warp per (sequence, group) row. Lane l keeps the running top list of blocks
+// l, l + 32, l + 64, ... (ascending, so the 32-bit insertion keeps the tie rule); the 32 lane
+// lists are then merged in KM rounds, each taking the warp's best head by the full key
+// (score, then lower block id) and advancing the winning lane's list.
+template <int KM>
+__global__ void __launch_bounds__(256) topk_decode_kernel(const __grid_constant__ TopkDecodeParams P) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= P.B * P.G) return;
+  const int b = row / P.G;
+  const int L = P.seqlens[b];
+  int32_t* out = P.block_ids + static_cast<int64_t>(row) * P.k;
+  if (L < 1 || (L - 1) / 128 >= P.nbmax) {  // host validated lmax; guard anyway
+    if (lane == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidTopk);
+    for (int s = lane; s < P.k; s += 32) out[s] = -1;
+    return;
+  }
+  const int bl = (L - 1) / 128;
+  if (bl + 1 <= P.k) {
+    if (lane == 0) topk_all_visible(bl, P.k, out);
+    return;
+  }
+  if constexpr (KM == 0) {   // k = 1: the local block alone
+    if (lane == 0) out[0] = bl;
+  } else {
+  const uint32_t* src = P.maxima + static_cast<int64_t>(row) * P.nbmax;
+  uint32_t Ls[KM];
+  int Lb[KM];
+#pragma unroll
+  for (int p = 0; p < KM; ++p) { Ls[p] = 0u; Lb[p] = -1; }
+  for (int kb = lane; kb < bl; kb += 32) topk_insert_ascending<KM>(Ls, Lb, __ldg(src + kb), kb);
+  int ids[KM];
+#pragma unroll
+  for (int r = 0; r < KM; ++r) {
+    // this lane's head as a 64-bit key (0 when its list is exhausted: below every real key)
+    uint64_t key = (Lb[0] >= 0) ? ((static_cast<uint64_t>(Ls[0]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(Lb[0])))
+                                : 0ull;
+    uint64_t best = key;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
+    ids[r] = static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(best));
+    if (key == best) {   // keys are unique (distinct block ids): exactly one lane advances
+#pragma unroll
+      for (int p = 0; p + 1 < KM; ++p) { Ls[p] = Ls[p + 1]; Lb[p] = Lb[p + 1]; }
+      Ls[KM - 1] = 0u;
+      Lb[KM - 1] = -1;
+    }
+  }
+  // odd-even transposition sort, ascending (the same on every lane)
+#pragma unroll
+  for (int pass = 0; pass < KM; ++pass) {
+#pragma unroll
+    for (int p = pass & 1; p + 1 < KM; p += 2) {
+      const int a = ids[p], c = ids[p + 1];
+      ids[p] = min(a, c);
+      ids[p + 1] = max(a, c);
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int p = 0; p < KM; ++p) out[p] = ids[p];
+    out[KM] = bl;
+  }
+  }
+}
+
 // 16-byte asynchronous global -> shared copy (bypassing L1); with ok == false nothing is
 // read and the 16 shared bytes are zero-filled. Both addresses 16-byte aligned.
 __device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc, bool ok) {

@@ -270,7 +270,7 @@ msa_status_t dispatch_topk_prefill(int k, const TopkPrefillParams& tp, dim3 grid
 template <int KM>
 void launch_topk_decode(const TopkDecodeParams& tp, cudaStream_t st) {
   const int rows = tp.B * tp.G;
-  topk_decode_kernel<KM><<<(rows + 127) / 128, 128, 0, st>>>(tp);
+  topk_decode_kernel<KM><<<(rows + 7) / 8, 256, 0, st>>>(tp);   // one warp per row
 }
 
 msa_status_t dispatch_topk_decode(int k, const TopkDecodeParams& tp, cudaStream_t st) {

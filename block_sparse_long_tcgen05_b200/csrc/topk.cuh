@@ -130,25 +130,4 @@ struct TopkDecodeParams {
   int B, G, k, nbmax;
 };
 
-// one thread per (sequence, group) row
-template <int KM>
-__global__ void __launch_bounds__(128) topk_decode_kernel(const __grid_constant__ TopkDecodeParams P) {
-  const int row = blockIdx.x * blockDim.x + threadIdx.x;
-  if (row >= P.B * P.G) return;
-  const int b = row / P.G;
-  const int L = P.seqlens[b];
-  int32_t* out = P.block_ids + static_cast<int64_t>(row) * P.k;
-  if (L < 1 || (L - 1) / 128 >= P.nbmax) {  // host validated lmax; guard anyway
-    record_error(MSA_ERR_DEVICE_BOUNDS, kKidTopk);
-    for (int s = 0; s < P.k; ++s) out[s] = -1;
-    return;
-  }
-  const int bl = (L - 1) / 128;
-  if (bl + 1 <= P.k) {
-    topk_all_visible(bl, P.k, out);
-    return;
-  }
-  topk_select_row<KM>(P.maxima + static_cast<int64_t>(row) * P.nbmax, 1, bl, out);
-}
-
 }  // namespace msa
