@@ -197,15 +197,37 @@ struct DecodeAttnParams {
   float scale_log2;
 };
 
+// Warp-level tensor-core helpers (mma.sync m16n8k16, bf16 in, fp32 accumulate). The decode
+// products have M = R <= 16 query heads, too few rows for tcgen05 (M >= 64).
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(smem_u32(row_addr)));
+}
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t (&r)[2], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(smem_u32(row_addr)));
+}
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// One CTA (4 warps) per (sequence, group, slot): K / V of the selected block staged in shared
+// memory, S = Q K^T and O = P V on tensor cores (M = 16 rows: the group's R <= 16 heads, the
+// rest zero), the softmax per head in between. Fragment coordinates: lane = 4 * gq + tq.
 template <int D>
 __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant__ DecodeAttnParams P) {
-  constexpr int KS = D + 8;    // padded smem row (bank spread)
+  constexpr int KS = D + 8;    // padded smem row: the 8 rows of an ldmatrix hit distinct banks
   extern __shared__ uint8_t dsm[];
   __nv_bfloat16* Ks = reinterpret_cast<__nv_bfloat16*>(dsm);
   __nv_bfloat16* Vs = Ks + 128 * KS;
-  float* Qs = reinterpret_cast<float*>(Vs + 128 * KS);   // [R][D]
-  float* Ss = Qs + P.R * D;                              // [R][128]
-  float* stat = Ss + P.R * 128;                          // [R][2]: max, 1/sum
+  float* Ss = reinterpret_cast<float*>(Vs + 128 * KS);   // [R][128]: scores, then P
+  float* stat = Ss + P.R * 128;                          // [R][2]: max, sum
   const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int blk = P.block_ids[(static_cast<int64_t>(b) * P.G + g) * P.k + s];
   if (blk < 0) return;
@@ -218,11 +240,8 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
   const int j0 = blk * 128;
   const int nvalid = min(128, pos - j0 + 1);
   const int tid = threadIdx.x;
-  // q rows, pre-scaled into log2 units
-  for (int e = tid; e < P.R * D; e += 128) {
-    const int r = e / D, dd = e % D;
-    Qs[e] = __bfloat162float(P.q[(static_cast<int64_t>(b) * P.G * P.R + g * P.R + r) * D + dd]) * P.scale_log2;
-  }
+  const int warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;
   // K / V rows of the block, 16-byte asynchronous copies all in flight at once (rows past
   // the query are zero-filled: source size 0)
   constexpr int CPR = D / 8;
@@ -233,75 +252,98 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
     cp_async16(Ks + j * KS + c * 8, P.kc + off, ok);
     cp_async16(Vs + j * KS + c * 8, P.vc + off, ok);
   }
+  const __nv_bfloat16* q0 = P.q + (static_cast<int64_t>(b) * P.G * P.R + g * P.R) * D;   // head 0 of the group
+  const bool r_lo = gq < P.R, r_hi = gq + 8 < P.R;
+  auto qpair = [&](int r, int col) -> uint32_t { return *reinterpret_cast<const uint32_t*>(q0 + r * D + col); };
   cp_async_wait_all();
   __syncthreads();
-  // scores: thread = key
+  // ---- S = Q K^T: warp w takes keys [32 w, 32 w + 32) as four 8-key tiles
   {
-    const int j = tid;
-    for (int r = 0; r < P.R; ++r) {
-      float acc = 0.0f;
-      if (j < nvalid) {
-#pragma unroll 4
-        for (int c = 0; c < CPR; ++c) {
-          const uint4 raw = *reinterpret_cast<const uint4*>(Ks + j * KS + c * 8);
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    float acc[4][4];
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const float2 f = __bfloat1622float2(h2[t]);
-            acc = fmaf(Qs[r * D + c * 8 + 2 * t], f.x, acc);
-            acc = fmaf(Qs[r * D + c * 8 + 2 * t + 1], f.y, acc);
-          }
-        }
+    for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) acc[nt][x] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int k0 = kk * 16;
+      uint32_t a[4];
+      a[0] = r_lo ? qpair(gq, k0 + 2 * tq) : 0u;
+      a[1] = r_hi ? qpair(gq + 8, k0 + 2 * tq) : 0u;
+      a[2] = r_lo ? qpair(gq, k0 + 8 + 2 * tq) : 0u;
+      a[3] = r_hi ? qpair(gq + 8, k0 + 8 + 2 * tq) : 0u;
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt) {
+        const int n0 = warp * 32 + nt * 8;
+        uint32_t bf[2];   // keys n0 .. n0 + 7; dims k0 .. k0 + 7 (matrix 0) and k0 + 8 .. (matrix 1)
+        ldsm_x2(bf, Ks + (n0 + (lane & 7)) * KS + k0 + 8 * ((lane >> 3) & 1));
+        mma_16816(acc[nt], a, bf);
       }
-      Ss[r * 128 + j] = (j < nvalid) ? acc : -INFINITY;
+    }
+    // scores in log2 units; keys past the query -> -inf
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int n = warp * 32 + nt * 8 + 2 * tq;
+      if (r_lo) {
+        Ss[gq * 128 + n] = (n < nvalid) ? acc[nt][0] * P.scale_log2 : -INFINITY;
+        Ss[gq * 128 + n + 1] = (n + 1 < nvalid) ? acc[nt][1] * P.scale_log2 : -INFINITY;
+      }
+      if (r_hi) {
+        Ss[(gq + 8) * 128 + n] = (n < nvalid) ? acc[nt][2] * P.scale_log2 : -INFINITY;
+        Ss[(gq + 8) * 128 + n + 1] = (n + 1 < nvalid) ? acc[nt][3] * P.scale_log2 : -INFINITY;
+      }
     }
   }
   __syncthreads();
-  // softmax per head: warp w takes heads w, w + 4, ...
-  {
-    const int w = tid >> 5, lane = tid & 31;
-    for (int r = w; r < P.R; r += 4) {
-      float v4[4];
-      float mx = -INFINITY;
+  // softmax per head: warp w takes heads w, w + 4, ...; P = 2^(x - max) overwrites the scores
+  for (int r = warp; r < P.R; r += 4) {
+    float v4[4];
+    float mx = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) { v4[u] = Ss[r * 128 + lane + 32 * u]; mx = fmaxf(mx, v4[u]); }
+    for (int u = 0; u < 4; ++u) { v4[u] = Ss[r * 128 + lane + 32 * u]; mx = fmaxf(mx, v4[u]); }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float sum = 0.0f;
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.0f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) { v4[u] = exp2f(v4[u] - mx); sum += v4[u]; Ss[r * 128 + lane + 32 * u] = v4[u]; }
+    for (int u = 0; u < 4; ++u) { v4[u] = exp2f(v4[u] - mx); sum += v4[u]; Ss[r * 128 + lane + 32 * u] = v4[u]; }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      if (lane == 0) { stat[2 * r] = mx; stat[2 * r + 1] = sum; }
-    }
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) { stat[2 * r] = mx; stat[2 * r + 1] = sum; }
   }
   __syncthreads();
   const int64_t slot = (static_cast<int64_t>(b) * P.G + g) * P.k + s;
-  // O = P V: task (r, c) = head r, 8 columns c*8 .. c*8 + 7; 16-byte V loads, keys in order
-  for (int e = tid; e < P.R * CPR; e += 128) {
-    const int r = e / CPR, c = e % CPR;
-    float acc[8];
+  // ---- O = P V (P as bf16): warp w takes dims [w D / 4, (w + 1) D / 4) as D / 32 tiles of 8
+  {
+    constexpr int NT = D / 32;
+    float acc[NT][4];
 #pragma unroll
-    for (int x = 0; x < 8; ++x) acc[x] = 0.0f;
-#pragma unroll 4
-    for (int j = 0; j < nvalid; ++j) {
-      const float w = Ss[r * 128 + j];
-      const uint4 raw = *reinterpret_cast<const uint4*>(Vs + j * KS + c * 8);
-      acc[0] = fmaf(w, bf16lo(raw.x), acc[0]);
-      acc[1] = fmaf(w, bf16hi(raw.x), acc[1]);
-      acc[2] = fmaf(w, bf16lo(raw.y), acc[2]);
-      acc[3] = fmaf(w, bf16hi(raw.y), acc[3]);
-      acc[4] = fmaf(w, bf16lo(raw.z), acc[4]);
-      acc[5] = fmaf(w, bf16hi(raw.z), acc[5]);
-      acc[6] = fmaf(w, bf16lo(raw.w), acc[6]);
-      acc[7] = fmaf(w, bf16hi(raw.w), acc[7]);
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int x = 0; x < 4; ++x) acc[nt][x] = 0.0f;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const int k0 = kk * 16;
+      uint32_t a[4];
+      a[0] = r_lo ? pack_bf16x2(Ss[gq * 128 + k0 + 2 * tq], Ss[gq * 128 + k0 + 2 * tq + 1]) : 0u;
+      a[1] = r_hi ? pack_bf16x2(Ss[(gq + 8) * 128 + k0 + 2 * tq], Ss[(gq + 8) * 128 + k0 + 2 * tq + 1]) : 0u;
+      a[2] = r_lo ? pack_bf16x2(Ss[gq * 128 + k0 + 8 + 2 * tq], Ss[gq * 128 + k0 + 9 + 2 * tq]) : 0u;
+      a[3] = r_hi ? pack_bf16x2(Ss[(gq + 8) * 128 + k0 + 8 + 2 * tq], Ss[(gq + 8) * 128 + k0 + 9 + 2 * tq]) : 0u;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n0 = warp * (D / 4) + nt * 8;
+        uint32_t bf[2];   // keys k0 .. k0 + 7 (matrix 0) and k0 + 8 .. k0 + 15 (matrix 1), dims n0 .. n0 + 7
+        ldsm_x2_trans(bf, Vs + (k0 + (lane & 15)) * KS + n0);
+        mma_16816(acc[nt], a, bf);
+      }
     }
-    uint4 out;
-    out.x = pack_bf16x2(acc[0], acc[1]);
-    out.y = pack_bf16x2(acc[2], acc[3]);
-    out.z = pack_bf16x2(acc[4], acc[5]);
-    out.w = pack_bf16x2(acc[6], acc[7]);
-    *reinterpret_cast<uint4*>(P.opart + (slot * P.R + r) * D + c * 8) = out;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int n = warp * (D / 4) + nt * 8 + 2 * tq;
+      if (r_lo)
+        *reinterpret_cast<uint32_t*>(P.opart + (slot * P.R + gq) * D + n) = pack_bf16x2(acc[nt][0], acc[nt][1]);
+      if (r_hi)
+        *reinterpret_cast<uint32_t*>(P.opart + (slot * P.R + gq + 8) * D + n) = pack_bf16x2(acc[nt][2], acc[nt][3]);
+    }
   }
   if (tid < P.R) P.ml[slot * P.R + tid] = make_float2(stat[2 * tid], stat[2 * tid + 1]);
 }

@@ -836,7 +836,7 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   ap.k = p->k;
   ap.Lmax = p->lmax;
   ap.scale_log2 = scale * 1.4426950408889634f;
-  const int smem = 2 * 128 * (p->d + 8) * 2 + R * p->d * 4 + R * 128 * 4 + R * 8;
+  const int smem = 2 * 128 * (p->d + 8) * 2 + R * 128 * 4 + R * 8;
   const dim3 agrid(p->k, p->g, B);
   if (p->d == 128) {
     static std::once_flag once;
