@@ -212,6 +212,19 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       int Lb[KM];
 #pragma unroll
       for (int p = 0; p < KM; ++p) { Ls[p] = 0u; Lb[p] = -1; }
+      // Blocks that beat the list's current last entry wait in a 4-entry buffer (ascending
+      // block order) and go into the list together when some row of the warp has 4: the
+      // insertion network, which the whole warp runs whenever any row needs it, then runs
+      // about as often as the busiest row has candidates instead of whenever any row has one.
+      uint32_t cu[4];
+      int cb[4];
+      int nc = 0;
+      auto flush = [&]() {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          if (c < nc) topk_insert_ascending<KM>(Ls, Lb, cu[c], cb[c]);
+        nc = 0;
+      };
       for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
         const int ab = static_cast<int>(ik & 1);
         const uint32_t au = static_cast<uint32_t>(ik >> 1);
@@ -240,7 +253,13 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           m = __fadd_rn(m, 0.0f);   // -0 -> +0 so equal scores give equal keys
           uint32_t u = __float_as_uint(m);
           u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-          topk_insert_ascending<KM>(Ls, Lb, u, kb);
+          if (u > Ls[KM - 1]) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              if (nc == c) { cu[c] = u; cb[c] = kb; }
+            ++nc;
+          }
+          if (__any_sync(0xffffffffu, nc == 4)) flush();
         } else {
           tc_fence_before();
           __syncwarp();
@@ -248,6 +267,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
       }
       if (!ok || !tile_present) continue;
+      flush();
       const int64_t i = static_cast<int64_t>(qb) * 128 + row;
       if (i >= P.N) continue;
       int32_t* out = P.block_ids + (i * P.G + it.g) * P.k;
