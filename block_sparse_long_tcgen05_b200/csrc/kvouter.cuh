@@ -38,7 +38,7 @@
 
 namespace msa {
 
-constexpr int kKvItemTiles = 8;
+constexpr int kKvItemTiles = 4;
 constexpr int kKvQStages = 2;
 // Softmax warpgroups = S/P regions of TMEM (128 columns each). Tile n goes to warpgroup
 // n % kKvSoftmaxWGs. Two (the default): O is double-buffered and every thread may hold 128
