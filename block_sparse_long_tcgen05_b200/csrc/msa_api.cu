@@ -600,7 +600,7 @@ cudaStream_t aux_stream(int kind) {
 }
 cudaStream_t side_stream() { return aux_stream(0); }
 
-// Events of one call, released when the call returns (the driver frees them once they complete).
+// Events of one call, destroyed when the call returns (CUDA releases them once they complete).
 struct EventSet {
   std::vector<cudaEvent_t> ev;
   bool make(size_t n) {
