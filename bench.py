@@ -190,6 +190,40 @@ def timed(fn, steps: int, stream) -> float:
     return a.elapsed_time(b) / steps
 
 
+def stage_rates(stages: dict, cfg, peaks: dict) -> dict:
+    """Every prefill kernel's achieved rate against its own roofline, from the per-step stage
+    times: TFLOP/s of the score and attention products (fraction of the measured sustained
+    bf16 peak), GB/s of compulsory bytes for the HBM-bound passes (fraction of the measured
+    copy bandwidth). The CSR passes together move the block ids twice and write one entry per
+    (query, group, slot)."""
+    N, Hq, G, d, d_idx, Bk, k = cfg.N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.Bk, cfg.k
+    nb = (N + Bk - 1) // Bk
+    flops = {"index_topk": accounting.index_kernel_flops(0, nb, G, d_idx),
+             "index_blockmax": accounting.index_kernel_flops(0, nb, G, d_idx),
+             "kvouter": accounting.kvouter_flops(N, Hq, d, Bk, k)}
+    byts = dict(accounting.main_branch_bytes(N, Hq, G, d, Bk, k))
+    byts["topk_prefill"] = 4.0 * G * Bk * nb * (nb - 1) / 2 + 4.0 * N * G * k
+    out = {}
+    for name, v in stages.items():
+        sec = v["ms_per_step"] * 1e-3
+        if sec <= 0:
+            continue
+        r = {}
+        if name in flops:
+            r["tflops"] = flops[name] / sec / 1e12
+            r["frac_bf16_sustained"] = r["tflops"] / peaks["bf16_tflops_sustained"]
+        if name in byts:
+            r["gbs"] = byts[name] / sec / 1e9
+            r["frac_hbm"] = r["gbs"] / peaks["hbm_gbs"]
+        if r:
+            out[name] = r
+    csr_sec = sum(v["ms_per_step"] for n, v in stages.items() if n.startswith("csr")) * 1e-3
+    if csr_sec > 0:
+        gbs = 3.0 * 4 * N * G * k / csr_sec / 1e9
+        out["csr (all passes)"] = {"gbs": gbs, "frac_hbm": gbs / peaks["hbm_gbs"]}
+    return out
+
+
 def run_ours(args, world, rank, local):
     from block_sparse_long_tcgen05_b200 import msa
     msa.load_library()
@@ -285,6 +319,10 @@ def run_ours(args, world, rank, local):
                         "frac_measured_bf16_sustained": useful_tflops / peaks["bf16_tflops_sustained"],
                         "useful_tflop_per_step": (idx_f + main_f) / 1e12},
             "stages": stages, "roofline": roof, "gpu_launches": gpu_launches, "clocks": clk}
+    try:   # reporting only: a failure here must not cost the measurement
+        line["stage_rates"] = stage_rates(stages, rcfg, peaks)
+    except Exception as e:  # noqa: BLE001
+        line["stage_rates"] = {"error": repr(e)}
 
     # ------------------------------------------------ decode (query-stationary), same ranks
     if not args.no_decode:
