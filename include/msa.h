@@ -14,17 +14,18 @@
  *     order and are padded with -1.
  *   Main Branch, per query head h of group g = h / (Hq / G):
  *     o[i, h] = softmax(q[i, h] . k[j, g] * scale) . v[j, g] over the tokens j <= i of
- *     the selected blocks (standard scaled dot-product attention, scale 1/sqrt(d)
- *     unless given).
+ *     the selected blocks (scale 1/sqrt(d) unless given).
  *   Decode applies the same definition to one new query per sequence, at position
  *   seqlens[b] - 1 of that sequence's cache.
  *
  * Conventions for every entry point:
  *   - Tensors are row-major and contiguous, bf16 passed as raw 16-bit storage
  *     (const void*). Every pointer is a DEVICE pointer owned by the caller, 16-byte
- *     aligned. The library allocates and frees nothing; scratch memory comes from the
+ *     aligned, except the input and output buffers of msa_forward_host, which are host
+ *     memory. The library allocates and frees no memory; scratch memory comes from the
  *     caller's workspace (size from the matching *_workspace function; 256-byte
- *     aligned base).
+ *     aligned base). It keeps up to three extra streams per device of its own (see
+ *     msa_forward_host) and creates its events per call.
  *   - stream is a cudaStream_t (NULL = legacy default stream). All work is enqueued on
  *     it; no call synchronises the host, except msa_get_device_error.
  *   - Arguments are validated before anything is enqueued. A bad argument returns
