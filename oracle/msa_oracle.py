@@ -34,6 +34,16 @@ Readings where the pages are silent (each also listed in the design notes):
   * decode: the new token sits at position L-1 of its sequence, and the same
     definition is applied to that one query.
 
+Index-branch KL loss (hyper.ai page, Method, fourth paragraph; zhichai.net section 五.1):
+    5. For every (query i, group g), over the tokens T of the selected blocks (j <= i):
+       the Main Branch's group-averaged distribution P_main(j) = mean over the group's
+       heads of softmax_T(q[i,h] . k[j,g] * scale), the Index Branch's distribution
+       P_idx(j) = softmax_T(s_g(i, j) * idx_scale), and KL(P_main || P_idx) =
+       sum_j P_main(j) (log P_main(j) - log P_idx(j)) in natural log units. The pages leave
+       the index distribution's normalisation open; the readings taken here (softmax over
+       the selected tokens, idx_scale = 1 / sqrt(d_idx) by default, the Main Branch as the
+       target) are listed in the design notes.
+
 Precision. Scores are computed with an fp64 matrix product. When every index input
 is an integer (all the synthetic workloads), every partial sum is an integer below
 2**53, so the scores are exact and the selection is the exact one. The main branch
@@ -227,3 +237,48 @@ def decode_rows(inp: dict, seqs, Bk: int, k: int, scale: float | None = None):
             o_out[t, g * R:(g + 1) * R] = sdpa(qh[g * R:(g + 1) * R], to_f64(kc[toks, g, :]),
                                                to_f64(vc[toks, g, :]), sc)
     return ids_out, o_out
+
+
+# --------------------------------------------------------------------------------------
+# Index-branch KL loss (forward)
+# --------------------------------------------------------------------------------------
+
+def log_softmax(x: np.ndarray) -> np.ndarray:
+    """log softmax of a 1-D fp64 array (max-subtracted)."""
+    m = x.max()
+    return x - m - np.log(np.exp(x - m).sum())
+
+
+def index_kl_rows(q, k, q_idx, k_idx, block_ids: np.ndarray, rows, Bk: int, scale: float | None = None,
+                  idx_scale: float | None = None) -> np.ndarray:
+    """Step 5 for the given query rows: KL(P_main || P_idx) per (row, group), fp64.
+
+    q [N, Hq, d], k [N, G, d], q_idx / k_idx [N, G, d_idx] (torch or numpy), block_ids
+    [r, G, k] for the rows. The tokens are those the Main Branch attends (selected blocks,
+    j <= i); P_main averages the softmax of the group's heads, P_idx is the softmax of the
+    index scores over the same tokens.
+    """
+    rows = np.asarray(list(rows), dtype=np.int64)
+    N, Hq, d = q.shape
+    G, d_idx = k_idx.shape[1], k_idx.shape[2]
+    R = Hq // G
+    scale = (1.0 / np.sqrt(d)) if not scale else scale
+    idx_scale = (1.0 / np.sqrt(d_idx)) if not idx_scale else idx_scale
+    out = np.zeros((len(rows), G), dtype=np.float64)
+    for t, i in enumerate(rows):
+        i = int(i)
+        qi = to_f64(q[i])
+        qii = to_f64(q_idx[i])
+        for g in range(G):
+            toks = selected_tokens(block_ids[t, g], i, Bk)
+            tk = torch.as_tensor(toks) if isinstance(k, torch.Tensor) else toks
+            keys = to_f64(k[tk, g, :])
+            ikeys = to_f64(k_idx[tk, g, :])
+            p_main = np.zeros(len(toks), dtype=np.float64)
+            for h in range(g * R, (g + 1) * R):
+                p_main += np.exp(log_softmax((keys @ qi[h]) * scale))
+            p_main /= R
+            log_p_idx = log_softmax((ikeys @ qii[g]) * idx_scale)
+            nz = p_main > 0
+            out[t, g] = float(np.sum(p_main[nz] * (np.log(p_main[nz]) - log_p_idx[nz])))
+    return out

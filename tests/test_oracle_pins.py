@@ -193,12 +193,13 @@ def _dense_causal_gqa_torch(q, k, v):
     return o[0].permute(1, 0, 2).numpy()              # [N, Hq, d]
 
 
-@pytest.mark.parametrize("N,Hq,G,d", [(512, 8, 2, 64), (300, 6, 3, 32)])
-def test_dense_reduction_equals_causal_gqa(N, Hq, G, d):
+@pytest.mark.parametrize("N,Hq,G,d,Bk", [(512, 8, 2, 64, 128), (300, 6, 3, 32, 128), (300, 8, 2, 32, 64),
+                                          (200, 4, 2, 32, 32)])
+def test_dense_reduction_equals_causal_gqa(N, Hq, G, d, Bk):
     """Pin (a): with k * Bk covering the causal context every visible block is selected,
     and the Main Branch ('standard scaled dot-product attention' over the selected
-    tokens, hyper.ai page, Method) is dense causal GQA (torch SDPA, fp64)."""
-    Bk = 128
+    tokens, hyper.ai page, Method) is dense causal GQA (torch SDPA, fp64). Also at the
+    smaller block sizes of the block-size ablation (hyper.ai page, Experiment: 32, 64, 128)."""
     nb = -(-N // Bk)
     cfg, inp = _tiny_inputs(N=N, seed=31, Hq=Hq, G=G, d=d, k=nb)
     rows = list(range(N))
@@ -311,3 +312,103 @@ def test_lse_merge_identity():
     Lt = max(lses) + math.log(sum(math.exp(x - max(lses)) for x in lses))
     merged = sum(math.exp(x - Lt) * p for x, p in zip(lses, parts))
     np.testing.assert_allclose(merged, full, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("Bk", [32, 64])
+def test_block_size_refines_the_selection_consistently(Bk):
+    """Block sizes of the ablation (hyper.ai page, Experiment: 32, 64, 128). At Bk the pooled
+    score of a block equals the max of the pooled scores of its halves at Bk / 2 (a max over a
+    union), for every row and every non-local block; the local block of row i is i // Bk at
+    every size; and with k = 1 only the local block is kept."""
+    cfg, inp = _tiny_inputs(N=700, seed=53, Hq=4, G=2, d=32, k=4)
+    rows = [0, Bk - 1, Bk, 3 * Bk + 5, 699]
+    ids_a, sc_a = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, Bk, 4)
+    ids_h, sc_h = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, Bk // 2, 4)
+    for t, i in enumerate(rows):
+        for g in range(2):
+            A, H = sc_a[t][g], sc_h[t][g]
+            assert len(A) == i // Bk + 1 and len(H) == i // (Bk // 2) + 1
+            for b in range(len(A) - 1):
+                assert A[b] == max(H[2 * b], H[2 * b + 1])
+            assert i // Bk in ids_a[t, g]
+    ids1, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, Bk, 1)
+    assert [int(x) for x in ids1[:, 0, 0]] == [i // Bk for i in rows]
+
+
+# ------------------------------------------------------------------------------------
+# Index-branch KL loss (hyper.ai page, Method, fourth paragraph; zhichai.net section 五.1)
+# ------------------------------------------------------------------------------------
+
+def _kl_inputs(N=300, Hq=4, G=2, d=32, d_idx=32, seed=71, k=3):
+    cfg = synth.PrefillConfig("t", N=N, Hq=Hq, G=G, d=d, d_idx=d_idx, k=k, idx_range=3, seed=seed)
+    inp = synth.prefill_inputs(cfg)
+    return cfg, inp
+
+
+def test_kl_is_zero_when_the_index_head_mirrors_the_main_head():
+    """One head per group (R = 1), index query/key equal to the head's query/key and the same
+    scale: the two distributions coincide, so the KL is 0 on every row."""
+    cfg, inp = _kl_inputs(Hq=2, G=2)
+    rows = list(range(0, cfg.N, 7))
+    ids, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, 128, cfg.k)
+    kl = orc.index_kl_rows(inp["q"], inp["k"], inp["q"], inp["k"], ids, rows, 128,
+                           scale=0.3, idx_scale=0.3)
+    assert np.abs(kl).max() < 1e-12
+
+
+def test_kl_two_token_closed_form():
+    """Query 1 sees tokens {0, 1}: with a = mean over the group's heads of sigma(l_h0 - l_h1)
+    and b = sigma(c (y_0 - y_1)), KL = a ln(a / b) + (1 - a) ln((1 - a) / (1 - b)). With two
+    heads per group this also fixes the order of averaging (mean of the distributions, not of
+    per-head KLs) and the direction (Main Branch as the target)."""
+    cfg, inp = _kl_inputs(Hq=4, G=2, d=16, d_idx=8, seed=5)
+    ids, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], [1], 128, cfg.k)
+    kl = orc.index_kl_rows(inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], ids, [1], 128)
+    q = inp["q"].double().numpy()
+    k = inp["k"].double().numpy()
+    qi = inp["q_idx"].double().numpy()
+    ki = inp["k_idx"].double().numpy()
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    for g in range(2):
+        a = 0.0
+        for h in (2 * g, 2 * g + 1):
+            l0 = float(q[1, h] @ k[0, g]) / math.sqrt(16)
+            l1 = float(q[1, h] @ k[1, g]) / math.sqrt(16)
+            a += sig(l0 - l1) / 2
+        b = sig((float(qi[1, g] @ ki[0, g]) - float(qi[1, g] @ ki[1, g])) / math.sqrt(8))
+        want = a * math.log(a / b) + (1 - a) * math.log((1 - a) / (1 - b))
+        assert kl[0, g] == pytest.approx(want, rel=1e-12, abs=1e-14)
+        # the other direction differs on this input, so the test fixes it
+        other = b * math.log(b / a) + (1 - b) * math.log((1 - b) / (1 - a))
+        assert abs(other - want) > 1e-6
+
+
+def test_kl_uniform_main_branch_closed_form():
+    """Zero queries make every head's softmax uniform over the T selected tokens, so
+    KL = -ln T - (1/T) sum_j log P_idx(j), with log P_idx from scipy's logsumexp."""
+    from scipy.special import logsumexp
+    cfg, inp = _kl_inputs(N=400, Hq=4, G=2, d=32, d_idx=32, seed=9, k=2)
+    inp["q"] = torch.zeros_like(inp["q"])
+    rows = [0, 5, 130, 255, 399]
+    ids, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, 128, cfg.k)
+    kl = orc.index_kl_rows(inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], ids, rows, 128, idx_scale=0.25)
+    qi = inp["q_idx"].double().numpy()
+    ki = inp["k_idx"].double().numpy()
+    for t, i in enumerate(rows):
+        for g in range(2):
+            toks = [j for b in ids[t, g] if b >= 0 for j in range(b * 128, min(b * 128 + 128, i + 1))]
+            y = 0.25 * (ki[toks, g] @ qi[i, g])
+            logp = y - logsumexp(y)
+            want = -math.log(len(toks)) - float(np.mean(logp))
+            assert kl[t, g] == pytest.approx(want, rel=1e-10, abs=1e-12)
+
+
+def test_kl_nonnegative_and_zero_on_the_first_row():
+    """Gibbs' inequality on every row; query 0 sees one token, both distributions are the
+    same point mass."""
+    cfg, inp = _kl_inputs(N=600, Hq=8, G=2, d=32, d_idx=16, seed=13, k=2)
+    rows = list(range(0, 600, 11)) + [0]
+    ids, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, 128, cfg.k)
+    kl = orc.index_kl_rows(inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], ids, rows, 128)
+    assert kl.min() > -1e-12
+    assert np.abs(kl[-1]).max() < 1e-15
