@@ -9,10 +9,16 @@ scaling), or with --shard groups its range of GQA groups of one shared sequence 
 scaling); no data-path collective either way, the time is the max over ranks. Rank 0
 prints one JSON line. `--impl reference` times the fp64 CPU oracle on a bounded sample of query
 rows of the same workload instead (rank 0 only).
+
+At N = 1 the same line also reports every synthetic configuration (the 2K tiny prefill, 32K,
+128K, decode B = 64 x 128K and 1M) under "configs": tokens/s, useful TFLOP/s and its fraction
+of the measured bf16 peak, the HBM rate of the memory-bound kernels, and the oracle's
+per-query rate on the host cores beside it (--headline-only skips them).
 """
 from __future__ import annotations
 
 import argparse
+import ctypes
 import dataclasses
 import json
 import math
@@ -61,11 +67,16 @@ def kernel_sha256(kernel: str, csrc: str | None = None) -> str | None:
 
 
 def load_peaks():
+    """Roofline denominators: the measured HBM copy bandwidth, the measured cuBLAS bf16 burst
+    rate (the peak for kernels of a step of tens of milliseconds) and, as a labelled extra,
+    the seconds-long sustained rate with the SM clock it ran at."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
-    return dict(FALLBACK), "fallback"
+        out = {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}
+        out["sustained_sm_mhz"] = (d.get("clocks_under_load") or {}).get("sm_mhz_median")
+        return out, "measured"
+    return dict(FALLBACK, sustained_sm_mhz=None), "fallback"
 
 
 # ------------------------------------------------------------------------------ clocks
@@ -130,6 +141,29 @@ def oracle_sample(inp: dict, cfg, rows: int, seed: int):
     return rows / dt, dt
 
 
+def oracle_rows_rate(inp: dict, cfg, rows: int, seed: int):
+    """The oracle on `rows` seeded query rows of a prefill, reading the (device) inputs row by
+    row as the long-sequence parity tests do (no host copy of the whole sequence); returns
+    (query rows/s, seconds)."""
+    from oracle import msa_oracle as orc  # test / baseline infrastructure only
+    rng = np.random.default_rng(seed)
+    sel = sorted(rng.choice(cfg.N, size=min(rows, cfg.N), replace=False).tolist())
+    t0 = time.perf_counter()
+    ids, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], sel, cfg.Bk, cfg.k)
+    orc.attend_rows(inp["q"], inp["k"], inp["v"], ids, sel, cfg.Bk)
+    dt = time.perf_counter() - t0
+    return len(sel) / dt, dt
+
+
+def oracle_decode_rate(dinp: dict, dcfg, seqs: int):
+    """The oracle on the first `seqs` decode sequences; returns (new tokens/s, seconds)."""
+    from oracle import msa_oracle as orc  # test / baseline infrastructure only
+    t0 = time.perf_counter()
+    orc.decode_rows(dinp, range(seqs), dcfg.Bk, dcfg.k)
+    dt = time.perf_counter() - t0
+    return seqs / dt, dt
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -192,14 +226,14 @@ def timed(fn, steps: int, stream) -> float:
 
 def stage_rates(stages: dict, cfg, peaks: dict) -> dict:
     """Every prefill kernel's achieved rate against its own roofline, from the per-step stage
-    times: TFLOP/s of the score and attention products (fraction of the measured sustained
-    bf16 peak), GB/s of compulsory bytes for the HBM-bound passes (fraction of the measured
-    copy bandwidth). The CSR passes together move the block ids twice and write one entry per
+    times: TFLOP/s of the score and attention products (fraction of the measured bf16 burst
+    peak), GB/s of compulsory bytes for the HBM-bound passes (fraction of the measured copy
+    bandwidth). The CSR passes together move the block ids twice and write one entry per
     (query, group, slot)."""
     N, Hq, G, d, d_idx, Bk, k = cfg.N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.Bk, cfg.k
     nb = (N + Bk - 1) // Bk
-    flops = {"index_topk": accounting.index_kernel_flops(0, nb, G, d_idx),
-             "index_blockmax": accounting.index_kernel_flops(0, nb, G, d_idx),
+    flops = {"index_topk": accounting.index_kernel_flops(0, nb, G, d_idx, Bk),
+             "index_blockmax": accounting.index_kernel_flops(0, nb, G, d_idx, Bk),
              "kvouter": accounting.kvouter_flops(N, Hq, d, Bk, k)}
     byts = dict(accounting.main_branch_bytes(N, Hq, G, d, Bk, k))
     byts["topk_prefill"] = 4.0 * G * Bk * nb * (nb - 1) / 2 + 4.0 * N * G * k
@@ -211,7 +245,7 @@ def stage_rates(stages: dict, cfg, peaks: dict) -> dict:
         r = {}
         if name in flops:
             r["tflops"] = flops[name] / sec / 1e12
-            r["frac_bf16_sustained"] = r["tflops"] / peaks["bf16_tflops_sustained"]
+            r["frac_bf16_burst"] = r["tflops"] / peaks["bf16_tflops"]
         if name in byts:
             r["gbs"] = byts[name] / sec / 1e9
             r["frac_hbm"] = r["gbs"] / peaks["hbm_gbs"]
@@ -224,6 +258,244 @@ def stage_rates(stages: dict, cfg, peaks: dict) -> dict:
     return out
 
 
+def stage_table(stats: dict, steps: int) -> dict:
+    total = sum(v[1] for v in stats.values())
+    return {name: {"launches_per_step": launches / steps, "ms_per_step": tot / steps,
+                   "share": tot / total if total else None}
+            for name, (launches, tot) in sorted(stats.items(), key=lambda kv: -kv[1][1])}
+
+
+def roofline(stats: dict, steps: int, rcfg, peaks: dict, peak_src: str, traffic: dict, sm_mhz) -> dict:
+    """The dominant kernel's achieved rate: algorithmic work per launch over its average
+    launch time (CUDA events on the launching stream), against the measured burst peak of its
+    bound; the sustained bf16 figure and a clock-normalised rate are labelled extras."""
+    N = rcfg.N
+    nb = (N + rcfg.Bk - 1) // rcfg.Bk
+    dom = max(stats.items(), key=lambda kv: kv[1][1])[0]
+    dom_launches, dom_ms = stats[dom]
+    per_launch_s = dom_ms / dom_launches * 1e-3
+    launches_per_step = dom_launches / steps
+    traffic_b = traffic.get(dom) if traffic else None
+    if dom in ("index_blockmax", "index_topk", "kvouter"):
+        if dom == "kvouter":
+            work = accounting.kvouter_flops(N, rcfg.Hq, rcfg.d, rcfg.Bk, rcfg.k) / launches_per_step
+        else:
+            work = accounting.index_kernel_flops(0, nb, rcfg.G, rcfg.d_idx, rcfg.Bk) / launches_per_step
+        ach = work / per_launch_s / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "traffic": traffic_b,
+                "peak_source": f"{peak_src} bf16 burst (cuBLAS 8192^3, best of 10); of {peak_src}",
+                "work_per_launch": work,
+                "sustained_extra": {"peak": peaks["bf16_tflops_sustained"],
+                                    "frac": ach / peaks["bf16_tflops_sustained"],
+                                    "peak_sm_mhz": peaks.get("sustained_sm_mhz"),
+                                    "note": "seconds-long GEMM loop under the power cap, at a lower SM clock "
+                                            "than this step's"}}
+    else:
+        byts = accounting.main_branch_bytes(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.Bk, rcfg.k).get(dom, float("nan"))
+        work = byts / launches_per_step
+        ach = work / per_launch_s / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": ach / peaks["hbm_gbs"], "traffic": traffic_b,
+                "peak_source": f"{peak_src} HBM copy; of {peak_src}", "work_per_launch": work}
+    if sm_mhz:
+        roof["achieved_per_sm_ghz"] = ach / (sm_mhz / 1000.0)
+        roof["sm_mhz_median"] = sm_mhz
+    return roof
+
+
+def prefill_rates(rcfg, ms: float, peaks: dict, world: int) -> dict:
+    idx_f, main_f = accounting.prefill_useful_flops(rcfg.N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.d_idx, rcfg.Bk, rcfg.k)
+    tf = (idx_f + main_f) / (ms * 1e-3) / 1e12
+    return {"useful_tflops": tf * world, "useful_tflops_per_gpu": tf,
+            "frac_measured_bf16_burst": tf / peaks["bf16_tflops"],
+            "frac_spec_bf16_2250": tf / SPEC_BF16_TFLOPS,
+            "frac_measured_bf16_sustained_extra": tf / peaks["bf16_tflops_sustained"],
+            "useful_tflop_per_step": (idx_f + main_f) / 1e12}
+
+
+def memory_bound_rates(stages: dict, rcfg, peaks: dict) -> dict:
+    """HBM rate of the memory-bound stages of a prefill: the merge, the CSR build and the
+    Top-k (a separate pass only on the two-kernel Index Branch; the one-kernel path keeps it in
+    the score epilogue, with no block maxima in HBM)."""
+    sr = stage_rates(stages, rcfg, peaks)
+    out = {}
+    for name, key in (("merge", "merge"), ("csr", "csr (all passes)"), ("topk", "topk_prefill")):
+        if key in sr:
+            out[name] = {"gbs": sr[key]["gbs"], "frac_hbm": sr[key]["frac_hbm"]}
+    if "topk_prefill" not in stages and "index_topk" in stages:
+        out["topk"] = "fused into index_topk (no block maxima in HBM)"
+    return out
+
+
+def make_prefill(cfg, dev, seed, query_chunk, shard_groups: bool, world: int, rank: int):
+    """Inputs, parameters and buffers of one prefill configuration on this rank."""
+    from block_sparse_long_tcgen05_b200 import msa
+    if shard_groups:
+        full = synth.prefill_inputs(cfg, device=dev, seed=cfg.seed)
+        inp = mdist.shard_inputs_by_group(full, cfg.G, world, rank)
+        del full
+        torch.cuda.empty_cache()
+        groups, _, _ = mdist.group_slice(cfg.G, cfg.R, world, rank)
+        rcfg = dataclasses.replace(cfg, Hq=len(groups) * cfg.R, G=len(groups))
+    else:
+        inp = synth.prefill_inputs(cfg, device=dev, seed=seed)
+        rcfg = cfg
+    p = msa.prefill_params(cfg.N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.d_idx, rcfg.k, bk=rcfg.Bk, query_chunk=query_chunk)
+    bufs = {"ws": torch.empty(msa.msa_forward_workspace(p), dtype=torch.uint8, device=dev),
+            "o": torch.empty_like(inp["q"]),
+            "ids": torch.empty(cfg.N, rcfg.G, rcfg.k, dtype=torch.int32, device=dev)}
+    return inp, rcfg, p, bufs
+
+
+def time_prefill(inp, p, bufs, steps: int, warmup: int, stream, dev, world: int, clocks: bool):
+    """W untimed steps, then K timed steps between barriers; returns (ms per step as the max
+    over ranks, per-kernel stats of this rank, clock record or None)."""
+    from block_sparse_long_tcgen05_b200 import msa
+
+    def step():
+        msa.msa_forward(p, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], o=bufs["o"],
+                        block_ids=bufs["ids"], workspace=bufs["ws"])
+
+    for _ in range(warmup):
+        step()
+    msa.check_device_error(dev)
+    barrier(world)
+    sampler = ClockSampler(dev.index) if clocks else None
+    msa.msa_profile_start()
+    ms = timed(step, steps, stream)
+    stats = msa.msa_profile_stop()
+    clk = sampler.stop() if sampler else None
+    msa.check_device_error(dev)
+    ms = max_over_ranks(ms, world)
+    barrier(world)
+    return ms, stats, clk
+
+
+def run_decode(args, dev, stream, world, rank, peaks, cpu_baseline: bool) -> dict:
+    from block_sparse_long_tcgen05_b200 import msa
+    dcfg = synth.DEC128K
+    dinp = synth.decode_inputs(dcfg, device=dev, seed=mdist.rank_seed(dcfg.seed, rank))
+    dp = msa.decode_params(dcfg.B, dinp["k_cache"].shape[1], dinp["seqlens"], dcfg.Hq, dcfg.G, dcfg.d,
+                           dcfg.d_idx, dcfg.k)
+    dws = torch.empty(msa.msa_forward_workspace(dp), dtype=torch.uint8, device=dev)
+    do = torch.empty_like(dinp["q"])
+
+    def dstep():
+        msa.msa_forward(dp, dinp["q"], dinp["k_cache"], dinp["v_cache"], dinp["q_idx"],
+                        dinp["k_idx_cache"], o=do, workspace=dws)
+
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    msa.check_device_error(dev)
+    barrier(world)
+    msa.msa_profile_start()
+    dms = timed(dstep, args.steps, stream)
+    dstats = msa.msa_profile_stop()
+    msa.check_device_error(dev)
+    dms = max_over_ranks(dms, world)
+    barrier(world)
+    scan_ms = dstats.get("decode_scan", (1, float("nan")))[1] / args.steps
+    scan_bytes = accounting.decode_scan_bytes([dcfg.L] * dcfg.B, dcfg.G, dcfg.d_idx)
+    d_idx_f, d_main_f = accounting.decode_useful_flops([dcfg.L] * dcfg.B, dcfg.Hq, dcfg.G, dcfg.d,
+                                                       dcfg.d_idx, dcfg.Bk, dcfg.k)
+    tok_s = world * dcfg.B / (dms * 1e-3)
+    scan_gbs = scan_bytes / (scan_ms * 1e-3) / 1e9
+    out = {"workload": dcfg.name, "tokens_per_s": tok_s, "ms_per_step": dms,
+           "useful_tflops_per_gpu": (d_idx_f + d_main_f) / (dms * 1e-3) / 1e12,
+           "frac_measured_bf16_burst": (d_idx_f + d_main_f) / (dms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+           "scan_hbm_gbs": scan_gbs, "scan_frac_hbm": scan_gbs / peaks["hbm_gbs"],
+           "roofline": {"kernel": "decode_scan", "bound": "hbm", "achieved": scan_gbs, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": scan_gbs / peaks["hbm_gbs"],
+                        "work_per_launch": scan_bytes,
+                        "note": "a read-only stream against a read+write copy peak can read a little above 1"},
+           "stages": {k: {"ms_per_step": v[1] / args.steps} for k, v in dstats.items()}}
+    if cpu_baseline:
+        seqs = 2
+        rate, dt = oracle_decode_rate(dinp, dcfg, seqs)
+        out["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "us_per_query": 1e6 / rate,
+                               "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"{seqs} decode sequences of {dcfg.L} tokens (both branches, fp64), "
+                                         f"{dt:.1f} s"}
+        out["gpu_over_oracle"] = tok_s / rate
+    del dinp, dws, do
+    torch.cuda.empty_cache()
+    return out
+
+
+# oracle rows per configuration for the per-query rate (a few seconds of host time each)
+ORACLE_ROWS = {"prefill-2k-tiny": 256, "prefill-32k": 16, "prefill-128k": 16, "prefill-1m": 2}
+
+
+def config_report(cfg, dev, stream, args, peaks, rank) -> dict:
+    """One more prefill configuration at N = 1: tokens/s, useful TFLOP/s, fractions of the
+    measured bf16 burst peak, HBM rates of the memory-bound stages and the oracle's per-query
+    rate on the host cores."""
+    inp, rcfg, p, bufs = make_prefill(cfg, dev, cfg.seed, 0, False, 1, rank)
+    steps = args.steps if cfg.N <= 131072 else max(2, min(args.steps, 3))
+    ms, stats, _ = time_prefill(inp, p, bufs, steps, max(3, args.warmup), stream, dev, 1, False)
+    st = stage_table(stats, steps)
+    out = {"tokens_per_s": cfg.N / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
+           **prefill_rates(rcfg, ms, peaks, 1), "memory_bound": memory_bound_rates(st, rcfg, peaks),
+           "stages": {k: round(v["ms_per_step"], 4) for k, v in st.items()}}
+    if not args.no_cpu_baseline:
+        rate, dt = oracle_rows_rate(inp, cfg, ORACLE_ROWS.get(cfg.name, 4), seed=11)
+        out["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "us_per_query": 1e6 / rate,
+                               "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"{ORACLE_ROWS.get(cfg.name, 4)} seeded query rows of {cfg.name} "
+                                         f"(both branches, fp64, inputs read from the device row by row), "
+                                         f"{dt:.1f} s"}
+        out["gpu_over_oracle"] = out["tokens_per_s"] / rate
+    del inp, bufs
+    torch.cuda.empty_cache()
+    return out
+
+
+def kl_report(cfg, dev, stream, args, peaks) -> dict:
+    """The index-branch KL loss forward (msa_index_kl) on one configuration: per step one KL
+    pass over every (query, group), given the forward's block ids and log-sum-exp. Useful work:
+    per (query, head, selected token) 2 d FLOPs of logits, per (query, group, selected token)
+    2 d_idx FLOPs of index scores; the kernel's tensor work also counts the index product on
+    all R rows of a query (it repeats the index row per head) and whole blocks."""
+    from block_sparse_long_tcgen05_b200 import msa
+    inp, rcfg, p, bufs = make_prefill(cfg, dev, cfg.seed, 0, False, 1, 0)
+    lse = torch.empty(cfg.N, cfg.Hq, dtype=torch.float32, device=dev)
+    msa.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cfg.k, bk=cfg.Bk, block_ids=bufs["ids"],
+                lse=lse, o=bufs["o"], workspace=bufs["ws"])
+    kl = torch.empty(cfg.N, cfg.G, dtype=torch.float32, device=dev)
+    kp = msa.prefill_params(cfg.N, cfg.Hq, cfg.G, cfg.d, cfg.d_idx, cfg.k, bk=cfg.Bk)
+    kws = torch.empty(max(256, msa.load_library().msa_index_kl_workspace(ctypes.byref(kp))), dtype=torch.uint8,
+                      device=dev)
+
+    def step():
+        msa.index_kl(inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], bufs["ids"], lse, bk=cfg.Bk, kl=kl,
+                     workspace=kws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    msa.check_device_error(dev)
+    msa.msa_profile_start()
+    steps = max(3, min(args.steps, 10))
+    ms = timed(step, steps, stream)
+    stats = msa.msa_profile_stop()
+    msa.check_device_error(dev)
+    i = np.arange(cfg.N, dtype=np.int64)
+    sel = accounting._selected_tokens(i, cfg.Bk, cfg.k).sum()
+    useful = 2.0 * cfg.d * cfg.Hq * sel + 2.0 * cfg.d_idx * cfg.G * sel
+    nsel_blocks = float(np.minimum(i // cfg.Bk + 1, cfg.k).sum())
+    tensor = 2.0 * cfg.Bk * nsel_blocks * cfg.Hq * (cfg.d + cfg.d_idx)
+    kl_ms = stats.get("kl", (1, ms))[1] / steps
+    out = {"workload": cfg.name, "ms_per_step": ms, "steps": steps,
+           "useful_tflops": useful / (ms * 1e-3) / 1e12,
+           "kl_kernel": {"ms_per_step": kl_ms, "tensor_tflops": tensor / (kl_ms * 1e-3) / 1e12,
+                         "frac_bf16_burst": tensor / (kl_ms * 1e-3) / 1e12 / peaks["bf16_tflops"]},
+           "stages": {k: round(v[1] / steps, 4) for k, v in stats.items()},
+           "mean_kl_nats": float(kl.mean().item())}
+    del inp, bufs, lse, kl, kws
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args, world, rank, local):
     from block_sparse_long_tcgen05_b200 import msa
     msa.load_library()
@@ -232,137 +504,49 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream(dev)
     peaks, peak_src = load_peaks()
     cfg = synth.CONFIGS[args.workload]
-    if args.shard == "groups":
-        # one sequence for the whole job; this rank computes its contiguous range of groups
-        full = synth.prefill_inputs(cfg, device=dev, seed=cfg.seed)
-        inp = mdist.shard_inputs_by_group(full, cfg.G, world, rank)
-        del full
-        torch.cuda.empty_cache()
-        groups, _, _ = mdist.group_slice(cfg.G, cfg.R, world, rank)
-        rcfg = dataclasses.replace(cfg, Hq=len(groups) * cfg.R, G=len(groups))
-        seqs_per_job = 1
-        parallelism = f"GQA groups sharded over {world} GPU(s), one sequence, no collective"
-    else:
-        inp = synth.prefill_inputs(cfg, device=dev, seed=mdist.rank_seed(cfg.seed, rank))
-        rcfg = cfg
-        seqs_per_job = world
-        parallelism = "one independent sequence per GPU, no collective"
+    shard_groups = args.shard == "groups"
+    inp, rcfg, p, bufs = make_prefill(cfg, dev, mdist.rank_seed(cfg.seed, rank), args.query_chunk, shard_groups,
+                                      world, rank)
+    seqs_per_job = 1 if shard_groups else world
+    parallelism = (f"GQA groups sharded over {world} GPU(s), one sequence, no collective" if shard_groups
+                   else "one independent sequence per GPU, no collective")
     N = cfg.N
-    p = msa.prefill_params(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.d_idx, rcfg.k, query_chunk=args.query_chunk)
-    ws = torch.empty(msa.msa_forward_workspace(p), dtype=torch.uint8, device=dev)
-    o = torch.empty_like(inp["q"])
-    ids = torch.empty(N, rcfg.G, rcfg.k, dtype=torch.int32, device=dev)
-
-    def step():
-        msa.msa_forward(p, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], o=o, block_ids=ids,
-                        workspace=ws)
-
-    for _ in range(max(3, args.warmup)):
-        step()
-    msa.check_device_error(dev)
-    barrier(world)
-    clocks = ClockSampler(local) if rank == 0 else None
-    msa.msa_profile_start()
-    ms = timed(step, args.steps, stream)
-    stats = msa.msa_profile_stop()
-    clk = clocks.stop() if clocks else None
-    msa.check_device_error(dev)
-    ms = max_over_ranks(ms, world)
-    barrier(world)
-
-    idx_f, main_f = accounting.prefill_useful_flops(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.d_idx, rcfg.Bk, rcfg.k)
-    useful_tflops = (idx_f + main_f) / (ms * 1e-3) / 1e12
+    warmup = max(3, args.warmup)
+    ms, stats, clk = time_prefill(inp, p, bufs, args.steps, warmup, stream, dev, world, rank == 0)
     value = seqs_per_job * N / (ms * 1e-3)   # tokens of the whole job over the slowest rank's time
-
-    # per-kernel breakdown (this rank, same timed region)
-    stages = {}
-    total_stage_ms = sum(v[1] for v in stats.values())
-    for name, (launches, tot) in sorted(stats.items(), key=lambda kv: -kv[1][1]):
-        stages[name] = {"launches_per_step": launches / args.steps, "ms_per_step": tot / args.steps,
-                        "share": tot / total_stage_ms if total_stage_ms else None}
+    stages = stage_table(stats, args.steps)
     gpu_launches = sum(v[0] for v in stats.values())
-    nb = (N + 127) // 128
-    dom = max(stats.items(), key=lambda kv: kv[1][1])[0]
-    dom_launches, dom_ms = stats[dom]
-    per_launch_ms = dom_ms / dom_launches
-    traffic = args.traffic.get(dom) if args.traffic else None
-    if dom in ("index_blockmax", "index_topk"):
-        work = accounting.index_kernel_flops(0, nb, rcfg.G, rcfg.d_idx) / (dom_launches / args.steps)
-        ach = work / (per_launch_ms * 1e-3) / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 sustained (kernel timed inside a long step)",
-                "work_per_launch": work}
-    elif dom == "kvouter":
-        work = accounting.kvouter_flops(N, rcfg.Hq, rcfg.d, rcfg.Bk, rcfg.k) / (dom_launches / args.steps)
-        ach = work / (per_launch_ms * 1e-3) / 1e12
-        roof = {"kernel": dom, "bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops_sustained"],
-                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops_sustained"], "traffic": traffic,
-                "peak_source": f"{peak_src} bf16 sustained", "work_per_launch": work}
-    else:
-        byts = accounting.main_branch_bytes(N, rcfg.Hq, rcfg.G, rcfg.d, rcfg.Bk, rcfg.k).get(dom, float("nan"))
-        work = byts / (dom_launches / args.steps)
-        ach = work / (per_launch_ms * 1e-3) / 1e9
-        roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": ach / peaks["hbm_gbs"], "traffic": traffic, "peak_source": f"{peak_src} HBM copy",
-                "work_per_launch": work}
+    rates = prefill_rates(rcfg, ms, peaks, world)
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "strong" if args.shard == "groups" else "weak",
+            "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "strong" if shard_groups else "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded counter-based generator)",
             "config": workload_config(cfg, {"parallelism": parallelism}),
-            "prefill": {"tokens_per_s": value, "useful_tflops": useful_tflops * world,
-                        "useful_tflops_per_gpu": useful_tflops,
-                        "frac_spec_bf16_2250": useful_tflops / SPEC_BF16_TFLOPS,
-                        "frac_measured_bf16_burst": useful_tflops / peaks["bf16_tflops"],
-                        "frac_measured_bf16_sustained": useful_tflops / peaks["bf16_tflops_sustained"],
-                        "useful_tflop_per_step": (idx_f + main_f) / 1e12},
-            "stages": stages, "roofline": roof, "gpu_launches": gpu_launches, "clocks": clk}
+            "prefill": {"tokens_per_s": value, **rates},
+            "stages": stages,
+            "roofline": roofline(stats, args.steps, rcfg, peaks, peak_src, args.traffic,
+                                 clk.get("sm_mhz") if clk else None),
+            "gpu_launches": gpu_launches, "clocks": clk}
+    if clk and clk.get("sm_mhz"):
+        line["prefill"]["useful_tflops_per_sm_ghz"] = rates["useful_tflops_per_gpu"] / (clk["sm_mhz"] / 1000.0)
     try:   # reporting only: a failure here must not cost the measurement
         line["stage_rates"] = stage_rates(stages, rcfg, peaks)
+        line["prefill"]["memory_bound"] = memory_bound_rates(stages, rcfg, peaks)
     except Exception as e:  # noqa: BLE001
         line["stage_rates"] = {"error": repr(e)}
 
     # ------------------------------------------------ decode (query-stationary), same ranks
     if not args.no_decode:
-        dcfg = synth.DEC128K
-        dinp = synth.decode_inputs(dcfg, device=dev, seed=mdist.rank_seed(dcfg.seed, rank))
-        dp = msa.decode_params(dcfg.B, dinp["k_cache"].shape[1], dinp["seqlens"], dcfg.Hq, dcfg.G, dcfg.d,
-                               dcfg.d_idx, dcfg.k)
-        dws = torch.empty(msa.msa_forward_workspace(dp), dtype=torch.uint8, device=dev)
-        do = torch.empty_like(dinp["q"])
-
-        def dstep():
-            msa.msa_forward(dp, dinp["q"], dinp["k_cache"], dinp["v_cache"], dinp["q_idx"],
-                            dinp["k_idx_cache"], o=do, workspace=dws)
-
-        for _ in range(max(3, args.warmup)):
-            dstep()
-        msa.check_device_error(dev)
-        barrier(world)
-        msa.msa_profile_start()
-        dms = timed(dstep, args.steps, stream)
-        dstats = msa.msa_profile_stop()
-        dms = max_over_ranks(dms, world)
-        scan_ms = dstats.get("decode_scan", (1, float("nan")))[1] / args.steps
-        scan_bytes = accounting.decode_scan_bytes([dcfg.L] * dcfg.B, dcfg.G, dcfg.d_idx)
-        d_idx_f, d_main_f = accounting.decode_useful_flops([dcfg.L] * dcfg.B, dcfg.Hq, dcfg.G, dcfg.d,
-                                                           dcfg.d_idx, dcfg.Bk, dcfg.k)
-        line["decode"] = {"workload": dcfg.name, "tokens_per_s": world * dcfg.B / (dms * 1e-3),
-                          "ms_per_step": dms, "useful_tflops_per_gpu": (d_idx_f + d_main_f) / (dms * 1e-3) / 1e12,
-                          "scan_hbm_gbs": scan_bytes / (scan_ms * 1e-3) / 1e9,
-                          "scan_frac_hbm": scan_bytes / (scan_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                          "stages": {k: {"ms_per_step": v[1] / args.steps} for k, v in dstats.items()}}
-        del dinp, dws, do
-        torch.cuda.empty_cache()
+        line["decode"] = run_decode(args, dev, stream, world, rank, peaks,
+                                    cpu_baseline=(world == 1 and not args.no_cpu_baseline))
 
     # ------------------------------------------------ end to end from pinned host memory
     if not args.no_e2e:
         # msa_forward_host: page-locked host inputs in, host output back; the library pipelines
         # the copies with the kernels chunk by chunk (all copies inside the timed region)
         host = {n: t.cpu().pin_memory() for n, t in inp.items()}
-        o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        o_h = torch.empty(bufs["o"].shape, dtype=bufs["o"].dtype, pin_memory=True)
         h2d = sum(t.numel() * t.element_size() for t in host.values())
         d2h = o_h.numel() * o_h.element_size()
         dbuf = torch.empty(msa.msa_forward_host_device_bytes(p), dtype=torch.uint8, device=dev)
@@ -374,7 +558,7 @@ def run_ours(args, world, rank, local):
         estep()
         torch.cuda.synchronize(dev)
         msa.check_device_error(dev)
-        same = bool(torch.equal(o_h, o.cpu()))   # the same kernels on the same inputs: identical
+        same = bool(torch.equal(o_h, bufs["o"].cpu()))   # the same kernels on the same inputs: identical
         barrier(world)
         esteps = max(2, min(args.steps, 10))
         ems = max_over_ranks(timed(estep, esteps, stream), world)
@@ -390,6 +574,41 @@ def run_ours(args, world, rank, local):
         line["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"{args.ref_rows * 2} seeded query rows of {cfg.name} "
                                           f"(both branches, fp64), {dt:.1f} s"}
+
+    # ------------------------------------------------ the other synthetic configurations (N = 1)
+    if world == 1 and not args.headline_only:
+        headline = {"tokens_per_s": value, "ms_per_step": ms, "steps": args.steps, **rates,
+                    "memory_bound": line["prefill"].get("memory_bound"),
+                    "stages": {k: round(v["ms_per_step"], 4) for k, v in stages.items()}}
+        if "cpu_baseline" in line:
+            headline["cpu_baseline"] = dict(line["cpu_baseline"], us_per_query=1e6 / line["cpu_baseline"]["value"])
+            headline["gpu_over_oracle"] = value / line["cpu_baseline"]["value"]
+        del inp, bufs
+        torch.cuda.empty_cache()
+        configs = {}
+        for name in ("prefill-2k-tiny", "prefill-32k", "prefill-128k", "decode-b64-128k", "prefill-1m"):
+            try:
+                if name == cfg.name:
+                    configs[name] = headline
+                elif name == "decode-b64-128k":
+                    configs[name] = line.get("decode") or run_decode(args, dev, stream, 1, rank, peaks,
+                                                                     not args.no_cpu_baseline)
+                else:
+                    configs[name] = config_report(synth.CONFIGS[name], dev, stream, args, peaks, rank)
+            except Exception as e:  # noqa: BLE001  (reporting only)
+                configs[name] = {"error": repr(e)}
+        line["configs"] = configs
+        # the block-size ablation's efficiency side (Bk = 64, 32 at the 128K shapes) and the KL loss
+        for bk in (64, 32):
+            c = dataclasses.replace(synth.P128K, name=f"prefill-128k-bk{bk}", Bk=bk)
+            try:
+                line.setdefault("block_sizes", {})[c.name] = config_report(c, dev, stream, args, peaks, rank)
+            except Exception as e:  # noqa: BLE001
+                line.setdefault("block_sizes", {})[c.name] = {"error": repr(e)}
+        try:
+            line["index_kl"] = kl_report(synth.P128K, dev, stream, args, peaks)
+        except Exception as e:  # noqa: BLE001
+            line["index_kl"] = {"error": repr(e)}
     if rank == 0:
         print(json.dumps(line), flush=True)
 
@@ -405,6 +624,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true",
+                    help="skip the report of the other synthetic configurations (N = 1)")
     ap.add_argument("--shard", choices=["sequences", "groups"], default="sequences",
                     help="N > 1: one independent sequence per GPU (weak scaling) or the GQA groups of one "
                          "sequence split over the GPUs (strong scaling); no collective either way")

@@ -12,37 +12,39 @@ namespace msa {
 // ------------------------------------------------------------------------------------
 // Decode, Index Branch: block maxima of the one new query per sequence against every
 // full block before its local block (query-stationary: the index-key cache streams
-// through once, 64 contiguous bytes per lane per load).
+// through once, 64 contiguous bytes per lane per load). Blocks hold bk in {32, 64, 128}
+// tokens; a CTA scans 128 tokens, i.e. 128 / bk blocks.
 // ------------------------------------------------------------------------------------
 struct DecodeScanParams {
   const __nv_bfloat16* q_idx;   // [B][G][DI]
   const __nv_bfloat16* k_idx;   // [B][Lmax][G][DI]
   const int32_t* seqlens;
   uint32_t* maxima;             // [B][G][nbmax]
-  int B, G, nbmax;
+  int B, G, nbmax, bk;
   int64_t Lmax;
 };
 
-// grid (nbmax, B), 256 threads: one CTA per (sequence, block). Needs G * DI / 32 to be
-// a power of two <= 32 (checked by the host).
+// grid (ceil(Lmax / 128), B), 256 threads: one CTA per (sequence, 128-token span). Needs
+// G * DI / 32 to be a power of two <= 32 (checked by the host).
 template <int DI>
 __global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant__ DecodeScanParams P) {
-  __shared__ uint32_t smax[32];
+  __shared__ uint32_t smax[128];   // [G][4]
   const int b = blockIdx.y, kb = blockIdx.x;
   const int L = P.seqlens[b];
   if (L < 1 || L > P.Lmax) {
     if (kb == 0 && threadIdx.x == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidDecodeScan);
     return;
   }
-  const int bl = (L - 1) / 128;
-  if (kb >= bl) return;
+  const int bl = (L - 1) / P.bk;                    // local block: only blocks before it are scanned
+  const int ntok = min(128, bl * P.bk - kb * 128);  // tokens of this span in those blocks
+  if (ntok <= 0) return;
   const int cpt = P.G * DI / 32;             // 64-byte chunks per token
   constexpr int LPG = DI / 32;               // lanes (chunks) per group
   const int lane = threadIdx.x & 31;
   const int w = lane % cpt;                  // constant per lane since cpt | 32
   const int g = w / LPG;
   const int qoff = (w % LPG) * 32;
-  if (threadIdx.x < 32) smax[threadIdx.x] = 0u;
+  if (threadIdx.x < 128) smax[threadIdx.x] = 0u;
   float qv[32];
   {
     const uint4* qp = reinterpret_cast<const uint4*>(P.q_idx + (static_cast<int64_t>(b) * P.G + g) * DI + qoff);
@@ -61,8 +63,8 @@ __global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant_
   __syncthreads();
   const uint4* base = reinterpret_cast<const uint4*>(P.k_idx + (static_cast<int64_t>(b) * P.Lmax + kb * 128) *
                                                                    P.G * DI);
-  const int nchunks = 128 * cpt;
-  float best = -INFINITY;
+  const int nchunks = ntok * cpt;
+  float best[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // per block of the span
   for (int c0 = threadIdx.x; c0 < nchunks; c0 += 256 * 2) {
     uint4 raw[2][4];
 #pragma unroll
@@ -86,17 +88,30 @@ __global__ void __launch_bounds__(256) decode_scan_kernel(const __grid_constant_
       }
 #pragma unroll
       for (int o = 1; o < LPG; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      if (c0 + h * 256 < nchunks) best = fmaxf(best, acc);
+      const int c = c0 + h * 256;
+      const int f = (c / cpt) / P.bk;   // block of the span holding this token
+#pragma unroll
+      for (int ff = 0; ff < 4; ++ff)
+        if (c < nchunks && ff == f) best[ff] = fmaxf(best[ff], acc);
     }
   }
   if ((lane % LPG) == 0) {
-    float m = __fadd_rn(best, 0.0f);
-    uint32_t u = __float_as_uint(m);
-    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    atomicMax(&smax[g], u);
+#pragma unroll
+    for (int ff = 0; ff < 4; ++ff) {
+      if (best[ff] == -INFINITY) continue;   // no token of that block in this lane's share
+      float m = __fadd_rn(best[ff], 0.0f);
+      uint32_t u = __float_as_uint(m);
+      u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+      atomicMax(&smax[g * 4 + ff], u);
+    }
   }
   __syncthreads();
-  if (threadIdx.x < P.G) P.maxima[(static_cast<int64_t>(b) * P.G + threadIdx.x) * P.nbmax + kb] = smax[threadIdx.x];
+  const int F = 128 / P.bk;
+  for (int e = threadIdx.x; e < P.G * F; e += blockDim.x) {
+    const int gg = e / F, ff = e % F;
+    const int blk = kb * F + ff;
+    if (blk < bl) P.maxima[(static_cast<int64_t>(b) * P.G + gg) * P.nbmax + blk] = smax[gg * 4 + ff];
+  }
 }
 
 // ------------------------------------------------------------------------------------
@@ -117,12 +132,12 @@ __global__ void __launch_bounds__(256) topk_decode_kernel(const __grid_constant_
   const int b = row / P.G;
   const int L = P.seqlens[b];
   int32_t* out = P.block_ids + static_cast<int64_t>(row) * P.k;
-  if (L < 1 || (L - 1) / 128 >= P.nbmax) {  // host validated lmax; guard anyway
+  if (L < 1 || (L - 1) / P.bk >= P.nbmax) {  // host validated lmax; guard anyway
     if (lane == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidTopk);
     for (int s = lane; s < P.k; s += 32) out[s] = -1;
     return;
   }
-  const int bl = (L - 1) / 128;
+  const int bl = (L - 1) / P.bk;
   if (bl + 1 <= P.k) {
     if (lane == 0) topk_all_visible(bl, P.k, out);
     return;
@@ -192,7 +207,7 @@ struct DecodeAttnParams {
   const int32_t* block_ids;     // [B][G][k]
   __nv_bfloat16* opart;         // [B][G][k][R][D]
   float2* ml;                   // [B][G][k][R]
-  int B, G, R, k;
+  int B, G, R, k, bk;
   int64_t Lmax;
   float scale_log2;
 };
@@ -233,12 +248,12 @@ __global__ void __launch_bounds__(128) decode_attn_kernel(const __grid_constant_
   if (blk < 0) return;
   const int L = P.seqlens[b];
   const int pos = L - 1;
-  if (L < 1 || L > P.Lmax || blk > pos / 128) {
+  if (L < 1 || L > P.Lmax || blk > pos / P.bk) {
     if (threadIdx.x == 0) record_error(MSA_ERR_DEVICE_BOUNDS, kKidDecodeAttn);
     return;
   }
-  const int j0 = blk * 128;
-  const int nvalid = min(128, pos - j0 + 1);
+  const int j0 = blk * P.bk;
+  const int nvalid = min(P.bk, pos - j0 + 1);   // rows past it (beyond the block or the query) stay zero
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int gq = lane >> 2, tq = lane & 3;

@@ -114,7 +114,7 @@ index_blockmax_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   uint64_t* acc_empty = acc_full + 2;               // [2]
   uint64_t* mma_done = acc_empty + 2;               // [1]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  WaitCtl* abort_flag = reinterpret_cast<WaitCtl*>(tmem_base_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -124,7 +124,7 @@ index_blockmax_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     for (int i = 0; i < kIdxStages; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
     mbar_init(mma_done, 1);
-    *abort_flag = 0;
+    wait_ctl_init(abort_flag);
     fence_mbar_init();
   }
   if (warp == 1) {

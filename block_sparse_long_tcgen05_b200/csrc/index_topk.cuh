@@ -12,10 +12,17 @@
 // epilogue thread sees every block of its row: it keeps the best k - 1 keys
 // (ordkey(block max) << 32 | ~kb: higher score first, lower block index among equals) in
 // registers and writes the row's block_ids when the item ends. No block maxima reach memory.
-// Items are ordered group-major (one group's index keys, N * d_idx * 2 bytes, stay in L2
-// while all CTAs work on it), with the pairs of successive groups in alternating cost order,
-// and dealt to CTAs in snake order (alternating direction every round) so the per-CTA sums
-// of cost stay even.
+// Items are ordered group-major (one group's index keys, N * d_idx * 2 bytes, are streamed
+// by all CTAs at once), with the pairs of successive groups in alternating cost order, and
+// dealt to CTAs in snake order (alternating direction every round) so the per-CTA sums of
+// cost stay even.
+//
+// Block sizes BK in {32, 64, 128}: the MMA tiles stay 128 x 128, so one 128-key tile holds
+// F = 128 / BK blocks and the epilogue takes F segment maxima per tile. A query row needs
+// every block before its own, and with F > 1 some of those lie in the key tile of the row's
+// own query tile (the diagonal tile): the items then also score that tile, and each row keeps
+// only the blocks b < floor(i / BK). Those blocks end before the row's own block, so no token
+// mask is needed.
 #pragma once
 #include "index_blockmax.cuh"
 #include "topk.cuh"
@@ -23,8 +30,8 @@
 namespace msa {
 
 struct IdxTopkParams {
-  int nb;              // query blocks of the sequence
-  int npairs;          // ceil(nb / 2)
+  int nt;              // 128-query tiles of the sequence
+  int npairs;          // ceil(nt / 2)
   int G, k;
   int64_t N;
   int32_t* block_ids;  // [N, G, k]
@@ -37,14 +44,15 @@ struct IdxTopkItem {
 // item t: group-major; within a group the pairs run in alternating directions (the last group
 // descending), so the cost of consecutive items never jumps and the list ends with the
 // cheapest items
-__device__ __forceinline__ IdxTopkItem idx_topk_item(const IdxTopkParams& P, int t) {
+// (diag = 1 when the diagonal key tile is scored, i.e. for block sizes below 128)
+__device__ __forceinline__ IdxTopkItem idx_topk_item(const IdxTopkParams& P, int t, int diag) {
   IdxTopkItem it;
   it.g = t / P.npairs;
   const int pr = t - it.g * P.npairs;
   const int p = ((P.G - 1 - it.g) & 1) ? pr : P.npairs - 1 - pr;
   it.qa = 2 * p;
-  it.has_b = (it.qa + 1 < P.nb) ? 1 : 0;
-  it.kbend = it.has_b ? it.qa + 1 : it.qa;
+  it.has_b = (it.qa + 1 < P.nt) ? 1 : 0;
+  it.kbend = (it.has_b ? it.qa + 1 : it.qa) + diag;
   return it;
 }
 
@@ -55,12 +63,15 @@ __device__ __forceinline__ int idx_topk_slot(int r, int total) {
   return t < total ? t : -1;
 }
 
-template <int DI, int KM>
+template <int DI, int KM, int BK>
 __global__ void __launch_bounds__(kIdxThreads, 1)
 index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ IdxTopkParams P) {
   using C = IdxCfg<DI>;
   static_assert(KM >= 1, "at least one non-local place");
+  static_assert(BK == 32 || BK == 64 || BK == 128, "block size");
+  constexpr int F = 128 / BK;               // blocks per 128-key tile
+  constexpr int kDiag = (F > 1) ? 1 : 0;    // the diagonal key tile holds needed blocks
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
@@ -72,7 +83,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t* acc_empty = acc_full + 2;               // [2]
   uint64_t* mma_done = acc_empty + 2;               // [1]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_slot + 1);
+  WaitCtl* abort_flag = reinterpret_cast<WaitCtl*>(tmem_base_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -82,7 +93,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int i = 0; i < kIdxStages; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
     mbar_init(mma_done, 1);
-    *abort_flag = 0;
+    wait_ctl_init(abort_flag);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -107,7 +118,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int r = 0; r < rounds && ok; ++r) {
         const int t = idx_topk_slot(r, total);
         if (t < 0) continue;
-        const IdxTopkItem it = idx_topk_item(P, t);
+        const IdxTopkItem it = idx_topk_item(P, t, kDiag);
         if (it.kbend == 0) continue;
         const int qbuf = n_item & 1;
         const uint32_t qu = static_cast<uint32_t>(n_item >> 1);
@@ -156,7 +167,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int r = 0; r < rounds && ok; ++r) {
         const int t = idx_topk_slot(r, total);
         if (t < 0) continue;
-        const IdxTopkItem it = idx_topk_item(P, t);
+        const IdxTopkItem it = idx_topk_item(P, t, kDiag);
         if (it.kbend == 0) continue;
         const int qbuf = n_item & 1;
         const uint32_t qu = static_cast<uint32_t>(n_item >> 1);
@@ -176,7 +187,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           const uint32_t k_addr = smem_u32(smem + C::kKOff + s * C::kTileBytes);
           const uint32_t d_a = tmem + ab * 256;
           const uint32_t d_b = d_a + 128;
-          const bool a_active = kb < it.qa;
+          const bool a_active = kb < it.qa + kDiag;
 #pragma unroll
           for (int kk = 0; kk < C::kKSteps; ++kk) {
             const uint32_t koff = (kk * 32) / C::kRowBytes * C::kPanelBytes + (kk * 32) % C::kRowBytes;
@@ -203,9 +214,11 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int r = 0; r < rounds && ok; ++r) {
       const int t = idx_topk_slot(r, total);
       if (t < 0) continue;
-      const IdxTopkItem it = idx_topk_item(P, t);
+      const IdxTopkItem it = idx_topk_item(P, t, kDiag);
       const int qb = it.qa + tile;
       const bool tile_present = (tile == 0) || it.has_b;
+      const int64_t i = static_cast<int64_t>(qb) * 128 + row;
+      const int bl = static_cast<int>(i / BK);   // this row's local block
       // running top list: ordered scores (descending) and their block ids; 0 is below every
       // real ordered score
       uint32_t Ls[KM];
@@ -225,14 +238,27 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           if (c < nc) topk_insert_ascending<KM>(Ls, Lb, cu[c], cb[c]);
         nc = 0;
       };
+      // offer block b with segment maximum m (blocks arrive in ascending order)
+      auto offer = [&](float m, int b, bool valid) {
+        m = __fadd_rn(m, 0.0f);   // -0 -> +0 so equal scores give equal keys
+        uint32_t u = __float_as_uint(m);
+        u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+        if (valid && u > Ls[KM - 1]) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (nc == c) { cu[c] = u; cb[c] = b; }
+          ++nc;
+        }
+        if (__any_sync(0xffffffffu, nc == 4)) flush();
+      };
       for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
         const int ab = static_cast<int>(ik & 1);
         const uint32_t au = static_cast<uint32_t>(ik >> 1);
         if (!mbar_wait(&acc_full[ab], au & 1, abort_flag, kKidIndexScore)) { ok = false; break; }
         tc_fence_after();
-        if (tile_present && kb < qb) {
+        if (tile_present && kb < qb + kDiag) {
           const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + ab * 256 + tile * 128;
-          // the whole 128-column row in one TMEM round trip, then 8 independent max chains
+          // the whole 128-column row in one TMEM round trip, then independent max chains
           uint32_t v[4][32];
 #pragma unroll
           for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, v[c]);
@@ -240,26 +266,32 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[ab]);
-          float m8[8];
+          if constexpr (F == 1) {
+            float m8[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) m8[j] = -INFINITY;
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int j = 0; j < 32; j += 2)
-              m8[(c * 16 + (j >> 1)) & 7] =
-                  max3f(m8[(c * 16 + (j >> 1)) & 7], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
-          float m = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-          m = __fadd_rn(m, 0.0f);   // -0 -> +0 so equal scores give equal keys
-          uint32_t u = __float_as_uint(m);
-          u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-          if (u > Ls[KM - 1]) {
+            for (int j = 0; j < 8; ++j) m8[j] = -INFINITY;
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-              if (nc == c) { cu[c] = u; cb[c] = kb; }
-            ++nc;
+#pragma unroll
+              for (int j = 0; j < 32; j += 2)
+                m8[(c * 16 + (j >> 1)) & 7] =
+                    max3f(m8[(c * 16 + (j >> 1)) & 7], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
+            offer(fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))),
+                  kb, true);
+          } else {
+            constexpr int CPS = BK / 32;     // 32-column chunks per block
+#pragma unroll
+            for (int f = 0; f < F; ++f) {
+              float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+              for (int c = f * CPS; c < (f + 1) * CPS; ++c)
+#pragma unroll
+                for (int j = 0; j < 32; j += 2)
+                  m4[(j >> 1) & 3] = max3f(m4[(j >> 1) & 3], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
+              const int b = kb * F + f;
+              offer(fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])), b, b < bl);
+            }
           }
-          if (__any_sync(0xffffffffu, nc == 4)) flush();
         } else {
           tc_fence_before();
           __syncwarp();
@@ -268,11 +300,10 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       if (!ok || !tile_present) continue;
       flush();
-      const int64_t i = static_cast<int64_t>(qb) * 128 + row;
       if (i >= P.N) continue;
       int32_t* out = P.block_ids + (i * P.G + it.g) * P.k;
-      if (qb + 1 <= P.k) {
-        topk_all_visible(qb, P.k, out);
+      if (bl + 1 <= P.k) {
+        topk_all_visible(bl, P.k, out);
       } else {
         int ids[KM];
 #pragma unroll
@@ -288,7 +319,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
 #pragma unroll
         for (int p = 0; p < KM; ++p) out[p] = ids[p];
-        out[KM] = qb;
+        out[KM] = bl;
       }
     }
   }

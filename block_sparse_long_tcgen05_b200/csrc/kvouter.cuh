@@ -5,14 +5,15 @@
 // KV-outer sparse attention keeps tensor cores busy under block-granular access and
 // handles skewed block popularity without atomic updates (zhichai.net section 4.2).
 //
-// A work item is (group g, block b, up to kKvItemTiles tiles of the queries that chose b).
+// A work item is (group g, block b, up to kKvItemTiles tiles of the queries that chose b);
+// blocks hold BK in {32, 64, 128} keys.
 // A tile holds TQ = 128 / RP queries; query q of the tile owns rows [q*RP, q*RP + R) of a
 // 128-row operand, RP = max(R, 8), so every query starts on an 8-row group.
 // Per tile, with K_b / V_b resident in shared memory:
-//   S = Q K_b^T          tcgen05.mma, M = 128 rows, N = 128 keys, K = d (SMEM x SMEM) -> TMEM
+//   S = Q K_b^T          tcgen05.mma, M = 128 rows, N = BK keys, K = d (SMEM x SMEM) -> TMEM
 //   m = rowmax(S) * scale * log2e;  P = exp2(S * scale * log2e - m)  (causal mask only where b
 //       is the query's own block), written back over S in TMEM as bf16;  l = rowsum(P)
-//   O = P V_b            tcgen05.mma, M = 128, N = d, K = 128 keys (TMEM x SMEM) -> TMEM
+//   O = P V_b            tcgen05.mma, M = 128, N = d, K = BK keys (TMEM x SMEM) -> TMEM
 //   the unnormalised O (bf16) and (m, l) go to the query's slot s; a later pass merges
 //   the k slots of every query (no atomics).
 //
@@ -31,7 +32,7 @@
 // TMEM: S/P regions at columns 128 * w, w < kKvSoftmaxWGs; O region(s) after them.
 //
 // Shared-memory layouts (all 128-byte swizzled, 1024-byte aligned):
-//   K, V: [panel][128 keys][128 B]                     (8-row group stride 1 KB, panel 16 KB)
+//   K, V: [panel][BK keys][128 B]                      (8-row group stride 1 KB, panel BK * 128 B)
 //   Q, O staging: [8-row group][panel][8 rows][128 B]  (8-row group stride kPanels KB, panel 1 KB)
 #pragma once
 #include "ptx.cuh"
@@ -54,15 +55,17 @@ static_assert(kKvSoftmaxWGs * 128 + kKvOBufs * 128 <= 512, "TMEM holds 512 colum
 constexpr int kKvEpiWarp = 4 + 4 * kKvSoftmaxWGs;   // first warp of the epilogue warpgroup
 constexpr int kKvThreads = 32 * (kKvEpiWarp + 4);
 
-template <int D, int RP>
+template <int D, int RP, int BK>
 struct KvCfg {
   static constexpr int kPanels = D / 64;
-  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kTileBytes = 128 * D * 2;         // a query (or staging) tile: 128 rows
+  static constexpr int kKvBytes = BK * D * 2;            // a K or V block
+  static constexpr int kKvPanel = BK * 128;              // one 64-column panel of a K or V block
   static constexpr int kGroupBytes = kPanels * 1024;     // one 8-row group, all panels
   static constexpr int TQ = 128 / RP;
   static constexpr int kKOff = 0;                        // 2 K buffers
-  static constexpr int kVOff = 2 * kTileBytes;           // 2 V buffers
-  static constexpr int kQOff = 4 * kTileBytes;           // kKvQStages query stages
+  static constexpr int kVOff = 2 * kKvBytes;             // 2 V buffers
+  static constexpr int kQOff = 4 * kKvBytes;             // kKvQStages query stages
   static constexpr int kStgOff = kQOff + kKvQStages * kTileBytes;   // O staging (one tile)
   static constexpr int kBarOff = kStgOff + kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
@@ -80,15 +83,17 @@ struct KvParams {
 
 // tensor maps:
 //   tm_q: 4-D view of q [N][Hq][D] as (64 elems, Hq heads, D/64 panels, N), box (64, 8, D/64, 1)
-//   tm_k, tm_v: 3-D view of k / v [N][G][D] as (D, G, N), box (64, 1, 128)
+//   tm_k, tm_v: 3-D view of k / v [N][G][D] as (D, G, N), box (64, 1, BK)
 //   tm_o: 4-D view of the partials [rows][R][D] as (64, R, D/64, rows),
 //         box (64, min(R, 8), R >= 8 ? D/64 : 1, 1)
-template <int D, int RP>
+template <int D, int RP, int BK>
 __global__ void __launch_bounds__(kKvThreads, 1)
 kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                const __grid_constant__ KvParams P) {
-  using C = KvCfg<D, RP>;
+  using C = KvCfg<D, RP, BK>;
+  static_assert(BK == 32 || BK == 64 || BK == 128, "block size");
+  constexpr int NCH = BK / 32;               // 32-column chunks of S per row
   constexpr int TQ = C::TQ;
   constexpr int QS = kKvQStages;
   extern __shared__ uint8_t smem_raw[];
@@ -109,7 +114,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint64_t* s_done = o_free + NO;           // all S products of the CTA complete
   uint64_t* pv_done = s_done + 1;           // all PV products of the CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  WaitCtl* abort_flag = reinterpret_cast<WaitCtl*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -123,7 +128,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     for (int i = 0; i < NO; ++i) { mbar_init(&o_full[i], 1); mbar_init(&o_free[i], 4); }
     mbar_init(s_done, 1);
     mbar_init(pv_done, 1);
-    *abort_flag = 0;
+    wait_ctl_init(abort_flag);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -154,14 +159,14 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int kb = ni & 1;
         const uint32_t ph = static_cast<uint32_t>(ni >> 1) & 1;
         if (!mbar_wait(&k_empty[kb], ph ^ 1, abort_flag, kKidKvOuter)) break;
-        mbar_arrive_expect_tx(&k_full[kb], C::kTileBytes);
+        mbar_arrive_expect_tx(&k_full[kb], C::kKvBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(smem + C::kKOff + kb * C::kTileBytes + p * 16384, &tm_k, &k_full[kb], p * 64, g, b * 128);
+          tma_load_3d(smem + C::kKOff + kb * C::kKvBytes + p * C::kKvPanel, &tm_k, &k_full[kb], p * 64, g, b * BK);
         ++kn;
         if (!mbar_wait(&v_empty[kb], ph ^ 1, abort_flag, kKidKvOuter)) break;
-        mbar_arrive_expect_tx(&v_full[kb], C::kTileBytes);
+        mbar_arrive_expect_tx(&v_full[kb], C::kKvBytes);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(smem + C::kVOff + kb * C::kTileBytes + p * 16384, &tm_v, &v_full[kb], p * 64, g, b * 128);
+          tma_load_3d(smem + C::kVOff + kb * C::kKvBytes + p * C::kKvPanel, &tm_v, &v_full[kb], p * 64, g, b * BK);
         ++vn;
       }
       // drain: the last K and V loads issued into each buffer must land before the CTA exits
@@ -175,6 +180,9 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // Lane q of the warp owns query q of the tile: it loads the CSR entry and issues that
     // query's boxes (RP / 8 boxes of 8 heads x all panels).
     if (lane == 0) tma_prefetch_desc(&tm_q);
+    // every query row of the chunk is gathered once per block it chose, by CTAs working on
+    // the same group at about the same time: keep the rows in L2 ahead of the streamed partials
+    const uint64_t keep = l2_policy_evict_last();
     int nt = 0;
     bool ok = true;
     int4 nxt = first_item;
@@ -198,7 +206,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           uint8_t* dst = smem + C::kQOff + qs * C::kTileBytes + lane * (RP / 8) * C::kGroupBytes;
 #pragma unroll
           for (int h8 = 0; h8 < RP / 8; ++h8)
-            tma_load_4d(dst + h8 * C::kGroupBytes, &tm_q, &q_full[qs], 0, g * P.R + h8 * 8, 0, e >> 5);
+            tma_load_4d_hint(dst + h8 * C::kGroupBytes, &tm_q, &q_full[qs], 0, g * P.R + h8 * 8, 0, e >> 5, keep);
         }
       }
     }
@@ -218,7 +226,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     //         has read O(n - NO) out of the same TMEM columns.
     if (lane == 0) {
       const bool is_s = (warp == 1);
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, true);
       int n = 0, ni = 0;
       bool ok = true;
@@ -229,8 +237,8 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int ntiles = (it.z + TQ - 1) / TQ;
         const int kb = ni & 1;
         const uint32_t ph = static_cast<uint32_t>(ni >> 1) & 1;
-        const uint32_t k_addr = smem_u32(smem + C::kKOff + kb * C::kTileBytes);
-        const uint32_t v_addr = smem_u32(smem + C::kVOff + kb * C::kTileBytes);
+        const uint32_t k_addr = smem_u32(smem + C::kKOff + kb * C::kKvBytes);
+        const uint32_t v_addr = smem_u32(smem + C::kVOff + kb * C::kKvBytes);
         if (!mbar_wait(is_s ? &k_full[kb] : &v_full[kb], ph, abort_flag, kKidKvOuter)) { ok = false; break; }
         for (int j = 0; j < ntiles; ++j, ++n) {
           const int w = n % NB;                                   // S/P region and warpgroup
@@ -251,7 +259,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t adesc =
                   smem_desc(q_addr + (kk >> 2) * 1024 + (kk & 3) * 32, 16, C::kGroupBytes, kLayoutSw128);
-              const uint64_t bdesc = smem_desc(k_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024, kLayoutSw128);
+              const uint64_t bdesc = smem_desc(k_addr + (kk >> 2) * C::kKvPanel + (kk & 3) * 32, 16, 1024, kLayoutSw128);
               umma_bf16(d_s, adesc, bdesc, idesc_s, kk > 0);
             }
             umma_commit(&q_empty[qs]);
@@ -267,8 +275,8 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t d_o = tmem + NB * 128 + ob * 128;
             const uint32_t a_p = tmem + w * 128;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk)
-              umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(v_addr + kk * 2048, 16384, 1024, kLayoutSw128), idesc_o,
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(v_addr + kk * 2048, C::kKvPanel, 1024, kLayoutSw128), idesc_o,
                            kk > 0);
             umma_commit(&sp_free[w]);
             umma_commit(&o_full[ob]);
@@ -293,6 +301,8 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     const uint32_t lane_base = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t o_row = smem_u32(smem + C::kStgOff) + (m >> 3) * C::kGroupBytes + (m & 7) * 128;
     if (lane == 0) tma_prefetch_desc(&tm_o);
+    // partials are read back only by the merge, after the whole chunk: evicted first
+    const uint64_t stream_out = l2_policy_evict_first();
     int nt = 0;
     bool fail = false;
     int4 nxt = first_item;
@@ -342,10 +352,11 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           const uint8_t* src = smem + C::kStgOff + qw * (RP / 8) * C::kGroupBytes;
           if (P.R >= 8) {
 #pragma unroll
-            for (int h8 = 0; h8 < RP / 8; ++h8) tma_store_4d(&tm_o, src + h8 * C::kGroupBytes, 0, h8 * 8, 0, row);
+            for (int h8 = 0; h8 < RP / 8; ++h8)
+              tma_store_4d_hint(&tm_o, src + h8 * C::kGroupBytes, 0, h8 * 8, 0, row, stream_out);
           } else {
 #pragma unroll
-            for (int p = 0; p < C::kPanels; ++p) tma_store_4d(&tm_o, src + p * 1024, 0, 0, p, row);
+            for (int p = 0; p < C::kPanels; ++p) tma_store_4d_hint(&tm_o, src + p * 1024, 0, 0, p, row, stream_out);
           }
           bulk_commit_group();
         }
@@ -391,21 +402,22 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           pref_nt = base ? nt + NB : -1;
           if (base) e_pref = __ldg(base + jn * TQ + q);
         }
-        const int limit = !valid ? -1 : ((b == (i >> 7)) ? (i & 127) : 127);   // keys c <= limit are visible
+        const int limit = !valid ? -1 : ((b == i / BK) ? (i % BK) : BK - 1);   // keys c <= limit are visible
         // warps whose rows all see the whole block skip the per-key mask
-        const bool whole = __all_sync(0xffffffffu, limit == 127);
+        const bool whole = __all_sync(0xffffffffu, limit == BK - 1);
         // ---- row max (pass 1 over S; two 32-column loads per TMEM wait, 4 independent chains)
         if (!mbar_wait(&s_full[wg], u & 1, abort_flag, kKidKvOuter)) { fail = true; break; }
         tc_fence_after();
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        constexpr int LPW = (NCH >= 2) ? 2 : 1;   // 32-column loads per TMEM wait
 #pragma unroll 1
-        for (int c = 0; c < 4; c += 2) {
-          uint32_t v[2][32];
-          tmem_ld32(t_s + c * 32, v[0]);
-          tmem_ld32(t_s + c * 32 + 32, v[1]);
+        for (int c = 0; c < NCH; c += LPW) {
+          uint32_t v[LPW][32];
+#pragma unroll
+          for (int h = 0; h < LPW; ++h) tmem_ld32(t_s + (c + h) * 32, v[h]);
           tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
+          for (int h = 0; h < LPW; ++h) {
             if (whole) {
 #pragma unroll
               for (int x = 0; x < 32; x += 2)
@@ -426,7 +438,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ---- P = exp2(S * scale * log2e - m), written over S as bf16 (pass 2)
         float l4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < NCH; ++c) {
           uint32_t v[32];
           tmem_ld32(t_s + c * 32, v);
           tmem_ld_wait();

@@ -20,6 +20,7 @@ struct MergeParams {
   const float2* ml;            // [rows][G][k][R]: (m_s, l_s)
   const int32_t* block_ids;    // [rows0 + rows][G][k] (absolute row index)
   __nv_bfloat16* o;            // [rows0 + rows][Hq][D]
+  float* lse;                  // optional [rows0 + rows][Hq]: log-sum-exp of the logits (natural log)
   int64_t row0, rows;
   int G, R, k;
 };
@@ -150,14 +151,14 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S.stages * S.stage_bytes);
   uint64_t* empty = full + S.stages;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + S.stages);
+  WaitCtl* abort_flag = reinterpret_cast<WaitCtl*>(empty + S.stages);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     for (int s = 0; s < S.stages; ++s) {
       mbar_init(&full[s], 1 + 32);          // expect_tx arrival + one arrival per producer lane
       mbar_init(&empty[s], kMergeGroupThreads / 32);   // the four warps of the unit's group
     }
-    *abort_flag = 0;
+    wait_ctl_init(abort_flag);
     fence_mbar_init();
   }
   __syncthreads();
@@ -234,6 +235,8 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
           if (lane < P.k) wt[lane * P.R + r] = (W > 0.0f) ? __fdividef(e, W) : 0.0f;
+          if (P.lse != nullptr && lane == 0)   // logits are in log2 units: scale back by ln 2
+            P.lse[(P.row0 + u / P.G) * (P.G * P.R) + (u % P.G) * P.R + r] = (M + log2f(W)) * 0.6931471805599453f;
         }
       }
       __syncwarp();

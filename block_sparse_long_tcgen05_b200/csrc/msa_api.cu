@@ -17,6 +17,7 @@
 #include "csr.cuh"
 #include "index_blockmax.cuh"
 #include "index_topk.cuh"
+#include "kl.cuh"
 #include "kvouter.cuh"
 #include "merge.cuh"
 #include "decode.cuh"
@@ -97,11 +98,18 @@ std::vector<std::pair<int, int>> index_chunks(int64_t nb, int G, size_t cap = kM
 
 bool supported_r(int R) { return R == 1 || R == 2 || R == 4 || R == 8 || R == 16; }
 
+// Longest sequence of the two-kernel Index Branch: one launch's key runs must fit the run
+// table passed to index_blockmax_kernel (kIdxMaxRuns runs of kIdxKbRun key blocks).
+constexpr int64_t kTwoKernelMaxBlocks = int64_t(kIdxMaxRuns) * kIdxKbRun;
+// Longest sequence of the Main Branch: the CSR build keeps one 128-bit membership mask per
+// key block of the chunk's causal range in shared memory (227 KB per CTA).
+constexpr int64_t kCsrMaxBlocks = (227 * 1024) / 16;
+
 msa_status_t check_common(int64_t n, int32_t g, int32_t bk, int32_t k) {
   if (n < 1 || n > kMaxN) return fail(MSA_ERR_INVALID_ARG, "n=%lld out of range [1, %lld]", (long long)n, (long long)kMaxN);
   if (g < 1 || g > 64) return fail(MSA_ERR_INVALID_ARG, "g=%d out of range [1, 64]", g);
   if (k < 1 || k > 32) return fail(MSA_ERR_UNSUPPORTED, "k=%d unsupported (1..32)", k);
-  if (bk != 128) return fail(MSA_ERR_UNSUPPORTED, "bk=%d unsupported (only 128)", bk);
+  if (bk != 128 && bk != 64 && bk != 32) return fail(MSA_ERR_UNSUPPORTED, "bk=%d unsupported (32, 64, 128)", bk);
   return MSA_OK;
 }
 
@@ -178,11 +186,12 @@ msa_status_t set_smem(K kernel, int bytes) {
 // ------------------------------- per-kernel timing -------------------------------
 enum ProfKind {
   kPIndex, kPTopkPrefill, kPCsrCount, kPCsrScan, kPCsrOffsets, kPCsrScatter, kPCsrItems, kPKvOuter, kPMerge,
-  kPDecodeScan, kPTopkDecode, kPDecodeAttn, kPIndexTopk, kPNumKinds
+  kPDecodeScan, kPTopkDecode, kPDecodeAttn, kPIndexTopk, kPKl, kPKlMerge, kPNumKinds
 };
 const char* const kProfNames[kPNumKinds] = {"index_blockmax", "topk_prefill", "csr_count", "csr_scan",
                                             "csr_offsets", "csr_scatter", "csr_items", "kvouter", "merge",
-                                            "decode_scan", "topk_decode", "decode_attn", "index_topk"};
+                                            "decode_scan", "topk_decode", "decode_attn", "index_topk", "kl",
+                                            "kl_merge"};
 struct ProfRec {
   int kind;
   cudaEvent_t a, b;
@@ -322,6 +331,8 @@ msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32
     auto kbend = [&](int p) { const int qa = qb0 + 2 * p; return (qa + 1 < qb1) ? qa + 1 : qa; };
     const int maxend = P.npairs > 0 ? kbend(P.npairs - 1) : 0;
     P.nruns = (maxend + kIdxKbRun - 1) / kIdxKbRun;
+    if (P.nruns > kIdxMaxRuns)   // excluded by check_index_n before anything is enqueued
+      return fail(MSA_ERR_UNSUPPORTED, "index launch needs %d key runs (at most %d)", P.nruns, kIdxMaxRuns);
     int acc = 0;
     for (int c = 0; c < P.nruns; ++c) {
       int p = 0;
@@ -357,36 +368,73 @@ msa_status_t launch_index(const void* q_idx, const void* k_idx, int64_t n, int32
 }
 
 // The one-kernel Index Branch (Top-k fused into the score epilogue, no block maxima in
-// memory) serves the common k and sequences whose per-group index keys stay L2-resident
-// while every CTA streams them; anything else takes the two-kernel path.
-constexpr int64_t kFusedIndexMaxN = 262144;
+// memory) serves the common k at every length: its CTAs sweep the key blocks of one group in
+// near lockstep (each item starts at key block 0, and the items of a round have nearly equal
+// lengths), so the key tiles they stream are shared through L2 even when the group's index
+// keys are larger than L2. Anything else takes the two-kernel path.
+#ifndef MSA_FUSED_INDEX_MAX_N
+#define MSA_FUSED_INDEX_MAX_N ((int64_t(1) << 26) - 1)
+#endif
+constexpr int64_t kFusedIndexMaxN = MSA_FUSED_INDEX_MAX_N;
 bool fused_index_ok(int64_t n, int32_t k) {
   return n <= kFusedIndexMaxN && (k == 4 || k == 8 || k == 16 || k == 32);
+}
+
+// Sequence-length limit of the Index Branch path that serves (n, k); checked before anything
+// is enqueued.
+msa_status_t check_index_n(int64_t n, int32_t bk, int32_t k) {
+  const int64_t nb = (n + 127) / 128;
+  if (bk != 128 && !fused_index_ok(n, k))
+    return fail(MSA_ERR_UNSUPPORTED, "bk=%d takes the one-kernel Index Branch only (k in 4, 8, 16, 32; got k=%d)", bk, k);
+  if (!fused_index_ok(n, k) && nb > kTwoKernelMaxBlocks)
+    return fail(MSA_ERR_UNSUPPORTED, "n=%lld with k=%d takes the two-kernel Index Branch, which serves at most %lld tokens",
+                (long long)n, k, (long long)(kTwoKernelMaxBlocks * 128));
+  return MSA_OK;
+}
+
+// Sequence-length limit of the Main Branch (CSR build); checked before anything is enqueued.
+msa_status_t check_attn_n(int64_t n, int32_t bk) {
+  const int64_t nb = (n + bk - 1) / bk;
+  if (nb > kCsrMaxBlocks)
+    return fail(MSA_ERR_UNSUPPORTED, "n=%lld with bk=%d: the Main Branch serves at most %lld blocks (%lld tokens)",
+                (long long)n, bk, (long long)kCsrMaxBlocks, (long long)(kCsrMaxBlocks * bk));
+  return MSA_OK;
 }
 
 size_t index_ws_bytes(int64_t n, int32_t g, int32_t k) {
   return fused_index_ok(n, k) ? kAlign : index_layout(nullptr, n, g).bytes;
 }
 
-template <int DI, int KM>
+template <int DI, int KM, int BK>
 msa_status_t launch_index_topk_km(const CUtensorMap& tq, const CUtensorMap& tk, const IdxTopkParams& P,
                                   cudaStream_t st) {
   using C = IdxCfg<DI>;
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
-  std::call_once(once, [] { attr = set_smem(index_topk_kernel<DI, KM>, C::kSmemBytes); });
+  std::call_once(once, [] { attr = set_smem(index_topk_kernel<DI, KM, BK>, C::kSmemBytes); });
   if (attr != MSA_OK) return attr;
   const int total = P.G * P.npairs;
   const int grid = std::min(num_sms(), total);
   ProfScope ps(kPIndexTopk, st);
-  index_topk_kernel<DI, KM><<<grid, kIdxThreads, C::kSmemBytes, st>>>(tq, tk, P);
+  index_topk_kernel<DI, KM, BK><<<grid, kIdxThreads, C::kSmemBytes, st>>>(tq, tk, P);
   MSA_CHECK_LAUNCH();
   return MSA_OK;
 }
 
+template <int DI, int BK>
+msa_status_t launch_index_topk_bk(const CUtensorMap& tq, const CUtensorMap& tk, const IdxTopkParams& P, int32_t k,
+                                  cudaStream_t st) {
+  switch (k) {
+    case 4: return launch_index_topk_km<DI, 3, BK>(tq, tk, P, st);
+    case 8: return launch_index_topk_km<DI, 7, BK>(tq, tk, P, st);
+    case 16: return launch_index_topk_km<DI, 15, BK>(tq, tk, P, st);
+    default: return launch_index_topk_km<DI, 31, BK>(tq, tk, P, st);
+  }
+}
+
 template <int DI>
 msa_status_t launch_index_topk(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t* block_ids,
-                               int32_t k, cudaStream_t st) {
+                               int32_t bk, int32_t k, cudaStream_t st) {
   using C = IdxCfg<DI>;
   const uint64_t row_stride = uint64_t(g) * DI * 2;
   CUtensorMap tq, tk;
@@ -396,29 +444,27 @@ msa_status_t launch_index_topk(const void* q_idx, const void* k_idx, int64_t n, 
   if ((s = make_map_3d(&tq, q_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
   if ((s = make_map_3d(&tk, k_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
   IdxTopkParams P{};
-  P.nb = int((n + 127) / 128);
-  P.npairs = (P.nb + 1) / 2;
+  P.nt = int((n + 127) / 128);
+  P.npairs = (P.nt + 1) / 2;
   P.G = g;
   P.k = k;
   P.N = n;
   P.block_ids = block_ids;
-  switch (k) {
-    case 4: return launch_index_topk_km<DI, 3>(tq, tk, P, st);
-    case 8: return launch_index_topk_km<DI, 7>(tq, tk, P, st);
-    case 16: return launch_index_topk_km<DI, 15>(tq, tk, P, st);
-    default: return launch_index_topk_km<DI, 31>(tq, tk, P, st);
-  }
+  if (bk == 128) return launch_index_topk_bk<DI, 128>(tq, tk, P, k, st);
+  if (bk == 64) return launch_index_topk_bk<DI, 64>(tq, tk, P, k, st);
+  return launch_index_topk_bk<DI, 32>(tq, tk, P, k, st);
 }
 
-msa_status_t run_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx, int32_t k,
-                              int32_t* block_ids, void* ws, cudaStream_t st) {
+msa_status_t run_index_select(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx, int32_t bk,
+                              int32_t k, int32_t* block_ids, void* ws, cudaStream_t st) {
   if (fused_index_ok(n, k)) {
     switch (d_idx) {
-      case 32: return launch_index_topk<32>(q_idx, k_idx, n, g, block_ids, k, st);
-      case 64: return launch_index_topk<64>(q_idx, k_idx, n, g, block_ids, k, st);
-      default: return launch_index_topk<128>(q_idx, k_idx, n, g, block_ids, k, st);
+      case 32: return launch_index_topk<32>(q_idx, k_idx, n, g, block_ids, bk, k, st);
+      case 64: return launch_index_topk<64>(q_idx, k_idx, n, g, block_ids, bk, k, st);
+      default: return launch_index_topk<128>(q_idx, k_idx, n, g, block_ids, bk, k, st);
     }
   }
+  if (bk != 128) return fail(MSA_ERR_UNSUPPORTED, "bk=%d needs the one-kernel Index Branch", bk);
   IndexLayout L = index_layout(ws, n, g);
   switch (d_idx) {
     case 32: return launch_index<32>(q_idx, k_idx, n, g, L, block_ids, k, st);
@@ -476,38 +522,70 @@ int merge_sm_count(int sms) {
 }
 
 struct AttnLayout {
-  int64_t chunk_blocks = 0;   // query blocks per chunk
+  int64_t chunk_tiles = 0;    // 128-query tiles per chunk
   int64_t chunks = 0;
   uint32_t *hist = nullptr, *totals = nullptr, *bstart = nullptr, *istart = nullptr;
   int32_t* entries = nullptr;
   int4* items = nullptr;
   void* opart[2] = {nullptr, nullptr};   // chunk c uses buffer c % 2 (one buffer for one chunk)
   float2* ml[2] = {nullptr, nullptr};
+  CsrChunkTable table{};                  // per-chunk regions of the inverted index
+  float* kl_part = nullptr;               // msa_index_kl: one chunk's (query, group, slot) partial sums
   size_t bytes = 0;
 };
 
 int rows_per_query(int R) { return R < 8 ? 8 : R; }
 
-AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, int32_t k, int64_t query_chunk) {
-  const int64_t nb = (n + 127) / 128;
+// Tiles per chunk: the requested query chunk (a multiple of 128; 0 = the default), raised if
+// needed so that the sequence has at most kCsrMaxChunks chunks.
+int64_t chunk_tiles(int64_t n, int64_t query_chunk) {
+  const int64_t nt = (n + 127) / 128;
+  int64_t cq = (query_chunk > 0 ? query_chunk : kDefaultQueryChunk) / 128;
+  cq = std::max<int64_t>(cq, (nt + kCsrMaxChunks - 1) / kCsrMaxChunks);
+  return std::max<int64_t>(1, std::min(cq, nt));
+}
+
+// kl = true: the layout of msa_index_kl (the inverted index and one chunk's KL partials
+// instead of the attention partials).
+AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t k,
+                       int64_t query_chunk, bool kl = false) {
+  const int64_t nt = (n + 127) / 128;
+  const int64_t nblocks = (n + bk - 1) / bk;
+  const int64_t bpt = 128 / bk;
   const int R = hq / g;
   const int TQ = 128 / rows_per_query(R);
-  int64_t cq = (query_chunk > 0 ? query_chunk : kDefaultQueryChunk) / 128;
-  cq = std::max<int64_t>(1, std::min(cq, nb));
   AttnLayout L;
-  L.chunk_blocks = cq;
-  L.chunks = (nb + cq - 1) / cq;
-  const int64_t rows = cq * 128;
-  const int64_t nbuck = int64_t(g) * nb;
-  const int64_t max_entries = rows * g * k;
-  const int64_t max_items = max_entries / (int64_t(TQ) * kKvItemTiles) + nbuck + 1;
+  L.chunk_tiles = chunk_tiles(n, query_chunk);
+  L.chunks = (nt + L.chunk_tiles - 1) / L.chunk_tiles;
+  int64_t hist = 0, buckets = 0, entries = 0, items = 0;
+  for (int64_t c = 0; c < L.chunks; ++c) {
+    const int64_t t0 = c * L.chunk_tiles, ntc = std::min(L.chunk_tiles, nt - t0);
+    const int64_t nbk = std::min(nblocks, (t0 + ntc) * bpt);
+    const int64_t rows = std::min(n, (t0 + ntc) * 128) - t0 * 128;
+    L.table.hist[c] = hist;
+    L.table.bucket[c] = buckets;
+    L.table.entry[c] = entries;
+    L.table.item[c] = items;
+    hist += int64_t(g) * nbk * ntc;
+    buckets += int64_t(g) * nbk;
+    entries += rows * g * k;
+    items += rows * g * k / (int64_t(TQ) * kKvItemTiles) + int64_t(g) * nbk + 1;
+  }
+  L.table.bucket[L.chunks] = buckets;
+  const int64_t rows = L.chunk_tiles * 128;
+  const int64_t max_entries = rows * g * k;   // of one chunk
   Carver cv(ws);
-  L.hist = static_cast<uint32_t*>(cv.take(size_t(nbuck) * cq * 4));
-  L.totals = static_cast<uint32_t*>(cv.take(size_t(nbuck) * 4));
-  L.bstart = static_cast<uint32_t*>(cv.take(size_t(nbuck + 1) * 4));
-  L.istart = static_cast<uint32_t*>(cv.take(size_t(nbuck + 1) * 4));
-  L.entries = static_cast<int32_t*>(cv.take(size_t(max_entries) * 4));
-  L.items = static_cast<int4*>(cv.take(size_t(max_items) * 16));
+  L.hist = static_cast<uint32_t*>(cv.take(size_t(hist) * 4));
+  L.totals = static_cast<uint32_t*>(cv.take(size_t(buckets) * 4));
+  L.bstart = static_cast<uint32_t*>(cv.take(size_t(buckets + L.chunks) * 4));
+  L.istart = static_cast<uint32_t*>(cv.take(size_t(buckets + L.chunks) * 4));
+  L.entries = static_cast<int32_t*>(cv.take(size_t(entries) * 4));
+  L.items = static_cast<int4*>(cv.take(size_t(items) * 16));
+  if (kl) {
+    L.kl_part = static_cast<float*>(cv.take(size_t(max_entries) * 32));
+    L.bytes = cv.off;
+    return L;
+  }
   const int nbuf = (L.chunks > 1 && merge_sm_count(num_sms()) > 0) ? 2 : 1;   // overlap needs two
   for (int i = 0; i < nbuf; ++i) {
     L.opart[i] = cv.take(size_t(max_entries) * R * d * 2);
@@ -518,25 +596,37 @@ AttnLayout attn_layout(void* ws, int64_t n, int32_t hq, int32_t g, int32_t d, in
   return L;
 }
 
-template <int D, int RP>
+template <int D, int RP, int BK>
 msa_status_t launch_kvouter(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                             const KvParams& kp, int grid, cudaStream_t st) {
-  using C = KvCfg<D, RP>;
+  using C = KvCfg<D, RP, BK>;
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
-  std::call_once(once, [] { attr = set_smem(kvouter_kernel<D, RP>, C::kSmemBytes); });
+  std::call_once(once, [] { attr = set_smem(kvouter_kernel<D, RP, BK>, C::kSmemBytes); });
   if (attr != MSA_OK) return attr;
   ProfScope ps(kPKvOuter, st);
-  kvouter_kernel<D, RP><<<grid, kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, kp);
+  kvouter_kernel<D, RP, BK><<<grid, kKvThreads, C::kSmemBytes, st>>>(tq, tk, tv, to, kp);
   MSA_CHECK_LAUNCH();
   return MSA_OK;
 }
 
-template <int D>
-msa_status_t dispatch_kvouter(int R, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+template <int D, int BK>
+msa_status_t dispatch_kvouter_r(int R, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const CUtensorMap& to, const KvParams& kp, int grid, cudaStream_t st) {
+  if (R <= 8) return launch_kvouter<D, 8, BK>(tq, tk, tv, to, kp, grid, st);
+  return launch_kvouter<D, 16, BK>(tq, tk, tv, to, kp, grid, st);
+}
+
+msa_status_t dispatch_kvouter(int d, int R, int bk, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                               const CUtensorMap& to, const KvParams& kp, int grid, cudaStream_t st) {
-  if (R <= 8) return launch_kvouter<D, 8>(tq, tk, tv, to, kp, grid, st);
-  return launch_kvouter<D, 16>(tq, tk, tv, to, kp, grid, st);
+  if (d == 128) {
+    if (bk == 128) return dispatch_kvouter_r<128, 128>(R, tq, tk, tv, to, kp, grid, st);
+    if (bk == 64) return dispatch_kvouter_r<128, 64>(R, tq, tk, tv, to, kp, grid, st);
+    return dispatch_kvouter_r<128, 32>(R, tq, tk, tv, to, kp, grid, st);
+  }
+  if (bk == 128) return dispatch_kvouter_r<64, 128>(R, tq, tk, tv, to, kp, grid, st);
+  if (bk == 64) return dispatch_kvouter_r<64, 64>(R, tq, tk, tv, to, kp, grid, st);
+  return dispatch_kvouter_r<64, 32>(R, tq, tk, tv, to, kp, grid, st);
 }
 
 // The streaming merge: a ring of shared-memory stages, each holding one (query, group) slab
@@ -632,20 +722,61 @@ struct SideJoin {
   }
 };
 
+// The inverted index of every query chunk, in five launches (see csr.cuh).
+msa_status_t build_csr(const AttnLayout& L, const int32_t* block_ids, int64_t n, int32_t g, int32_t bk, int32_t k,
+                       int TQ, cudaStream_t st) {
+  CsrParams cp{};
+  cp.block_ids = block_ids;
+  cp.N = n;
+  cp.G = g;
+  cp.k = k;
+  cp.bk = bk;
+  cp.bpt = 128 / bk;
+  cp.ntiles = int((n + 127) / 128);
+  cp.nblocks = int((n + bk - 1) / bk);
+  cp.ct = int(L.chunk_tiles);
+  cp.nchunks = int(L.chunks);
+  cp.tq = TQ;
+  cp.item_tiles = kKvItemTiles;
+  cp.hist = L.hist;
+  cp.totals = L.totals;
+  cp.bucket_start = L.bstart;
+  cp.item_start = L.istart;
+  cp.entries = L.entries;
+  cp.items = L.items;
+  const int64_t buckets = L.table.bucket[L.chunks];
+  const size_t bm_bytes = size_t(cp.nblocks) * 16;   // masks of the last tile (checked by check_attn_n)
+  if (bm_bytes > 227 * 1024) return fail(MSA_ERR_UNSUPPORTED, "sequence too long for the CSR build (%d blocks)", cp.nblocks);
+  const dim3 tiles(unsigned(cp.ntiles), unsigned(g));
+  { ProfScope ps(kPCsrCount, st); csr_count_kernel<<<tiles, 128, bm_bytes, st>>>(cp, L.table); }
+  MSA_CHECK_LAUNCH();
+  { ProfScope ps(kPCsrScan, st); csr_scan_kernel<<<unsigned((buckets + 7) / 8), 256, 0, st>>>(cp, L.table); }
+  MSA_CHECK_LAUNCH();
+  { ProfScope ps(kPCsrOffsets, st); csr_offsets_kernel<<<unsigned(L.chunks), 1024, 0, st>>>(cp, L.table); }
+  MSA_CHECK_LAUNCH();
+  { ProfScope ps(kPCsrScatter, st); csr_scatter_kernel<<<tiles, 128, bm_bytes, st>>>(cp, L.table); }
+  MSA_CHECK_LAUNCH();
+  { ProfScope ps(kPCsrItems, st); csr_items_kernel<<<unsigned((buckets + 255) / 256), 256, 0, st>>>(cp, L.table); }
+  MSA_CHECK_LAUNCH();
+  return MSA_OK;
+}
+
 // chunk_in (optional, one event per chunk): the caller's stream waits for chunk_in[c] before
-// chunk c's kernels (its query rows and the key/value rows up to its end must be resident).
+// chunk c's attention kernels (its query rows and the key/value rows up to its end must be
+// resident; the inverted index needs only the block ids).
 // chunk_out (optional): recorded after chunk c's merge, once o's rows of chunk c are final.
 msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const int32_t* block_ids, int64_t n,
-                             int32_t hq, int32_t g, int32_t d, int32_t k, float scale, void* o, void* ws,
+                             int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t k, float scale, void* o, void* ws,
                              int64_t query_chunk, cudaStream_t st, const cudaEvent_t* chunk_in = nullptr,
-                             const cudaEvent_t* chunk_out = nullptr) {
+                             const cudaEvent_t* chunk_out = nullptr, float* lse = nullptr) {
   msa_status_t s;
   if ((s = set_csr_smem()) != MSA_OK) return s;
   const int R = hq / g;
   const int RP = rows_per_query(R);
   const int TQ = 128 / RP;
-  AttnLayout L = attn_layout(ws, n, hq, g, d, k, query_chunk);
-  const int64_t nb = (n + 127) / 128;
+  AttnLayout L = attn_layout(ws, n, hq, g, d, bk, k, query_chunk);
+  const int64_t nt = (n + 127) / 128;
+  const int64_t nblocks = (n + bk - 1) / bk;
   if (scale == 0.0f) scale = 1.0f / std::sqrt(float(d));
   CUtensorMap tq, tk, tv, to[2];
   const uint64_t panels = uint64_t(d) / 64;
@@ -654,13 +785,13 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
                        {uint64_t(d) * 2, 128, uint64_t(hq) * d * 2}, {64, 8, uint32_t(panels), 1},
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
-  if ((s = make_map_3d(&tk, kk, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
+  if ((s = make_map_3d(&tk, kk, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, uint32_t(bk),
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
-  if ((s = make_map_3d(&tv, v, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, 128,
+  if ((s = make_map_3d(&tv, v, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, uint32_t(bk),
                        CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
     return s;
-  const int64_t slot_rows = L.chunk_blocks * 128 * g * k;
+  const int64_t slot_rows = L.chunk_tiles * 128 * g * k;
   // partials [rows][R][d] as (64 elems, R heads, panels, rows); R >= 8: one box per 8 heads
   // covering all panels, R < 8: one box per panel
   for (int i = 0; i < 2; ++i)
@@ -669,6 +800,7 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
                          {64, uint32_t(std::min(R, 8)), R >= 8 ? uint32_t(panels) : 1u, 1},
                          CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
       return s;
+  if ((s = build_csr(L, block_ids, n, g, bk, k, TQ, st)) != MSA_OK) return s;
   const int sms = num_sms();
   const int msms = (L.chunks > 1 && L.opart[1] != L.opart[0]) ? merge_sm_count(sms) : 0;
   cudaStream_t side = msms > 0 ? side_stream() : nullptr;
@@ -678,59 +810,28 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     return fail(MSA_ERR_CUDA, "cudaEventCreateWithFlags failed");
   SideJoin join;   // declared after the events: it runs first when the call returns
   if (overlap) { join.st = st; join.side = side; }
-  int64_t ci = 0;
-  for (int64_t qa0 = 0; qa0 < nb; qa0 += L.chunk_blocks, ++ci) {
-    const int64_t qa1 = std::min(nb, qa0 + L.chunk_blocks);
+  for (int64_t ci = 0; ci < L.chunks; ++ci) {
+    const int64_t t0 = ci * L.chunk_tiles, t1 = std::min(nt, t0 + L.chunk_tiles);
+    const int64_t nbk = std::min(nblocks, t1 * (128 / bk));
     const int buf = int(ci & 1);
     if (chunk_in && cudaStreamWaitEvent(st, chunk_in[ci], 0) != cudaSuccess)
       return fail(MSA_ERR_CUDA, "cudaStreamWaitEvent failed");
-    CsrParams cp{};
-    cp.block_ids = block_ids;
-    cp.N = n;
-    cp.G = g;
-    cp.k = k;
-    cp.qa0 = int(qa0);
-    cp.qa1 = int(qa1);
-    cp.nt = int(qa1 - qa0);
-    cp.tq = TQ;
-    cp.item_tiles = kKvItemTiles;
-    cp.hist = L.hist;
-    cp.totals = L.totals;
-    cp.bucket_start = L.bstart;
-    cp.item_start = L.istart;
-    cp.entries = L.entries;
-    cp.items = L.items;
-    const int64_t nbuck = int64_t(g) * qa1;
-    const size_t bm_bytes = size_t(qa1) * 16;
-    if (bm_bytes > 227 * 1024) return fail(MSA_ERR_UNSUPPORTED, "sequence too long for the CSR build (%lld blocks)", (long long)qa1);
-    { ProfScope ps(kPCsrCount, st); csr_count_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp); }
-    MSA_CHECK_LAUNCH();
-    { ProfScope ps(kPCsrScan, st); csr_scan_kernel<<<unsigned((nbuck + 7) / 8), 256, 0, st>>>(cp); }
-    MSA_CHECK_LAUNCH();
-    { ProfScope ps(kPCsrOffsets, st); csr_offsets_kernel<<<1, 1024, 0, st>>>(cp); }
-    MSA_CHECK_LAUNCH();
-    { ProfScope ps(kPCsrScatter, st); csr_scatter_kernel<<<dim3(cp.nt, g), 128, bm_bytes, st>>>(cp); }
-    MSA_CHECK_LAUNCH();
-    { ProfScope ps(kPCsrItems, st); csr_items_kernel<<<unsigned((nbuck + 255) / 256), 256, 0, st>>>(cp); }
-    MSA_CHECK_LAUNCH();
     KvParams kp{};
-    kp.entries = L.entries;
-    kp.items = L.items;
-    kp.n_items = L.istart + nbuck;
+    kp.entries = L.entries + L.table.entry[ci];
+    kp.items = L.items + L.table.item[ci];
+    kp.n_items = L.istart + L.table.bucket[ci] + ci + int64_t(g) * nbk;
     kp.G = g;
     kp.R = R;
     kp.k = k;
-    kp.nbk = int(qa1);
-    kp.row0 = qa0 * 128;
+    kp.nbk = int(nbk);
+    kp.row0 = t0 * 128;
     kp.scale_log2 = scale * 1.4426950408889634f;
     kp.ml = L.ml[buf];
     // buffer `buf` was last read by the merge of chunk ci - 2
     if (overlap && ci >= 2 && cudaStreamWaitEvent(st, m_done.ev[ci - 2], 0) != cudaSuccess)
       return fail(MSA_ERR_CUDA, "cudaStreamWaitEvent failed");
     const int kv_grid = (overlap && ci > 0) ? sms - msms : sms;
-    if (d == 128) s = dispatch_kvouter<128>(R, tq, tk, tv, to[buf], kp, kv_grid, st);
-    else s = dispatch_kvouter<64>(R, tq, tk, tv, to[buf], kp, kv_grid, st);
-    if (s != MSA_OK) return s;
+    if ((s = dispatch_kvouter(d, R, bk, tq, tk, tv, to[buf], kp, kv_grid, st)) != MSA_OK) return s;
     cudaStream_t mst = st;
     if (overlap) {
       if (cudaEventRecord(kv_done.ev[ci], st) != cudaSuccess || cudaStreamWaitEvent(side, kv_done.ev[ci], 0) != cudaSuccess)
@@ -742,8 +843,9 @@ msa_status_t run_sparse_attn(const void* q, const void* kk, const void* v, const
     mp.ml = L.ml[buf];
     mp.block_ids = block_ids;
     mp.o = static_cast<__nv_bfloat16*>(o);
-    mp.row0 = qa0 * 128;
-    mp.rows = std::min<int64_t>(n, qa1 * 128) - qa0 * 128;
+    mp.lse = lse;
+    mp.row0 = t0 * 128;
+    mp.rows = std::min<int64_t>(n, t1 * 128) - t0 * 128;
     mp.G = g;
     mp.R = R;
     mp.k = k;
@@ -768,7 +870,7 @@ struct DecodeLayout {
 
 DecodeLayout decode_layout(void* ws, const msa_params* p, bool need_ids) {
   const int64_t B = p->n;
-  const int64_t nbmax = (p->lmax + 127) / 128;
+  const int64_t nbmax = (p->lmax + p->bk - 1) / p->bk;
   const int R = p->hq / p->g;
   Carver cv(ws);
   DecodeLayout L;
@@ -785,7 +887,7 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   DecodeLayout L = decode_layout(ws, p, block_ids_out == nullptr);
   int32_t* ids = block_ids_out ? block_ids_out : L.block_ids;
   const int B = int(p->n);
-  const int nbmax = int((p->lmax + 127) / 128);
+  const int nbmax = int((p->lmax + p->bk - 1) / p->bk);
   const int R = p->hq / p->g;
   const float scale = p->scale == 0.0f ? 1.0f / std::sqrt(float(p->d)) : p->scale;
   DecodeScanParams sp{};
@@ -796,8 +898,9 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   sp.B = B;
   sp.G = p->g;
   sp.nbmax = nbmax;
+  sp.bk = p->bk;
   sp.Lmax = p->lmax;
-  const dim3 sgrid(nbmax, B);
+  const dim3 sgrid(unsigned((p->lmax + 127) / 128), B);
   {
     ProfScope ps(kPDecodeScan, st);
     switch (p->d_idx) {
@@ -816,6 +919,7 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   tp.G = p->g;
   tp.k = p->k;
   tp.nbmax = nbmax;
+  tp.bk = p->bk;
   msa_status_t s;
   {
     ProfScope ps(kPTopkDecode, st);
@@ -834,6 +938,7 @@ msa_status_t run_decode(const msa_params* p, const void* q, const void* kc, cons
   ap.G = p->g;
   ap.R = R;
   ap.k = p->k;
+  ap.bk = p->bk;
   ap.Lmax = p->lmax;
   ap.scale_log2 = scale * 1.4426950408889634f;
   const int smem = 2 * 128 * (p->d + 8) * 2 + R * 128 * 4 + R * 8;
@@ -890,6 +995,120 @@ msa_status_t check_d_idx(int32_t d_idx) {
 
 size_t prefill_ids_bytes(int64_t n, int32_t g, int32_t k) { return align_up(size_t(n) * g * k * 4); }
 
+// ------------------------------- index-branch KL loss -------------------------------
+template <int D, int BK, int DI>
+msa_status_t launch_kl(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tki, const KlParams& kp,
+                       int grid, cudaStream_t st) {
+  using C = KlCfg<D, 8, BK, DI>;
+  static std::once_flag once;
+  static msa_status_t attr = MSA_OK;
+  std::call_once(once, [] { attr = set_smem(kl_kernel<D, 8, BK, DI>, C::kSmemBytes); });
+  if (attr != MSA_OK) return attr;
+  ProfScope ps(kPKl, st);
+  kl_kernel<D, 8, BK, DI><<<grid, kKlThreads, C::kSmemBytes, st>>>(tq, tk, tki, kp);
+  MSA_CHECK_LAUNCH();
+  return MSA_OK;
+}
+
+template <int D, int BK>
+msa_status_t dispatch_kl_di(int di, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tki,
+                            const KlParams& kp, int grid, cudaStream_t st) {
+  if (di == 128) return launch_kl<D, BK, 128>(tq, tk, tki, kp, grid, st);
+  if (di == 64) return launch_kl<D, BK, 64>(tq, tk, tki, kp, grid, st);
+  return launch_kl<D, BK, 32>(tq, tk, tki, kp, grid, st);
+}
+
+msa_status_t dispatch_kl(int d, int bk, int di, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tki,
+                         const KlParams& kp, int grid, cudaStream_t st) {
+  if (d == 128) {
+    if (bk == 128) return dispatch_kl_di<128, 128>(di, tq, tk, tki, kp, grid, st);
+    if (bk == 64) return dispatch_kl_di<128, 64>(di, tq, tk, tki, kp, grid, st);
+    return dispatch_kl_di<128, 32>(di, tq, tk, tki, kp, grid, st);
+  }
+  if (bk == 128) return dispatch_kl_di<64, 128>(di, tq, tk, tki, kp, grid, st);
+  if (bk == 64) return dispatch_kl_di<64, 64>(di, tq, tk, tki, kp, grid, st);
+  return dispatch_kl_di<64, 32>(di, tq, tk, tki, kp, grid, st);
+}
+
+msa_status_t run_index_kl(const msa_params* p, const void* q, const void* kk, const void* q_idx, const void* k_idx,
+                          const int32_t* block_ids, const float* lse, float idx_scale, float* kl, void* ws,
+                          cudaStream_t st) {
+  msa_status_t s;
+  if ((s = set_csr_smem()) != MSA_OK) return s;
+  const int64_t n = p->n;
+  const int g = p->g, hq = p->hq, d = p->d, di = p->d_idx, bk = p->bk, k = p->k;
+  const int R = hq / g;
+  const AttnLayout L = attn_layout(ws, n, hq, g, d, bk, k, p->query_chunk, true);
+  const int64_t nt = (n + 127) / 128;
+  const int64_t nblocks = (n + bk - 1) / bk;
+  const float scale = p->scale == 0.0f ? 1.0f / std::sqrt(float(d)) : p->scale;
+  if (idx_scale == 0.0f) idx_scale = 1.0f / std::sqrt(float(di));
+  CUtensorMap tq, tk, tki;
+  const uint64_t panels = uint64_t(d) / 64;
+  if ((s = make_map_4d(&tq, q, {64, uint64_t(hq), panels, uint64_t(n)},
+                       {uint64_t(d) * 2, 128, uint64_t(hq) * d * 2}, {64, 8, uint32_t(panels), 1},
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  if ((s = make_map_3d(&tk, kk, d, g, n, uint64_t(d) * 2, uint64_t(g) * d * 2, 64, 1, uint32_t(bk),
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  const bool sw64 = (di == 32);
+  if ((s = make_map_3d(&tki, k_idx, di, g, n, uint64_t(di) * 2, uint64_t(g) * di * 2, sw64 ? 32 : 64, 1, uint32_t(bk),
+                       sw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B)) != MSA_OK)
+    return s;
+  if ((s = build_csr(L, block_ids, n, g, bk, k, 16, st)) != MSA_OK) return s;
+  const int sms = num_sms();
+  for (int64_t ci = 0; ci < L.chunks; ++ci) {
+    const int64_t t0 = ci * L.chunk_tiles, t1 = std::min(nt, t0 + L.chunk_tiles);
+    const int64_t nbk = std::min(nblocks, t1 * (128 / bk));
+    KlParams kp{};
+    kp.entries = L.entries + L.table.entry[ci];
+    kp.items = L.items + L.table.item[ci];
+    kp.n_items = L.istart + L.table.bucket[ci] + ci + int64_t(g) * nbk;
+    kp.q_idx = static_cast<const __nv_bfloat16*>(q_idx);
+    kp.lse = lse;
+    kp.G = g;
+    kp.R = R;
+    kp.k = k;
+    kp.nbk = int(nbk);
+    kp.row0 = t0 * 128;
+    kp.scale_log2 = scale * 1.4426950408889634f;
+    kp.idx_scale_log2 = idx_scale * 1.4426950408889634f;
+    kp.part = L.kl_part;
+    if ((s = dispatch_kl(d, bk, di, tq, tk, tki, kp, sms, st)) != MSA_OK) return s;
+    KlMergeParams mp{};
+    mp.part = L.kl_part;
+    mp.block_ids = block_ids;
+    mp.kl = kl;
+    mp.row0 = t0 * 128;
+    mp.rows = std::min<int64_t>(n, t1 * 128) - t0 * 128;
+    mp.G = g;
+    mp.k = k;
+    mp.idx_scale = idx_scale;
+    {
+      ProfScope ps(kPKlMerge, st);
+      kl_merge_kernel<<<unsigned((mp.rows * g + 255) / 256), 256, 0, st>>>(mp);
+    }
+    MSA_CHECK_LAUNCH();
+  }
+  return MSA_OK;
+}
+
+msa_status_t check_kl_params(const msa_params* p) {
+  msa_status_t s;
+  if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
+  if (p->mode != MSA_MODE_PREFILL) return fail(MSA_ERR_UNSUPPORTED, "msa_index_kl takes prefill shapes only");
+  if ((s = check_common(p->n, p->g, p->bk, p->k)) != MSA_OK) return s;
+  if ((s = check_main_dims(p->hq, p->g, p->d)) != MSA_OK) return s;
+  if ((s = check_d_idx(p->d_idx)) != MSA_OK) return s;
+  if ((s = check_attn_n(p->n, p->bk)) != MSA_OK) return s;
+  if (p->hq / p->g > 8) return fail(MSA_ERR_UNSUPPORTED, "msa_index_kl takes hq/g <= 8 (got %d)", p->hq / p->g);
+  if (!(p->scale >= 0.0f) || std::isinf(p->scale)) return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
+  if (p->query_chunk < 0 || p->query_chunk % 128 != 0)
+    return fail(MSA_ERR_INVALID_ARG, "query_chunk=%lld must be a non-negative multiple of 128", (long long)p->query_chunk);
+  return MSA_OK;
+}
+
 }  // namespace
 
 // =====================================================================================
@@ -913,7 +1132,7 @@ const char* msa_status_string(msa_status_t s) {
 const char* msa_last_error_detail(void) { return g_detail; }
 
 size_t msa_index_select_workspace(int64_t n, int32_t g, int32_t d_idx, int32_t bk, int32_t k) {
-  if (check_common(n, g, bk, k) != MSA_OK || check_d_idx(d_idx) != MSA_OK) return 0;
+  if (check_common(n, g, bk, k) != MSA_OK || check_d_idx(d_idx) != MSA_OK || check_index_n(n, bk, k) != MSA_OK) return 0;
   return index_ws_bytes(n, g, k);
 }
 
@@ -923,13 +1142,14 @@ msa_status_t msa_index_select(const void* q_idx, const void* k_idx, int64_t n, i
   msa_status_t s;
   if ((s = check_common(n, g, bk, k)) != MSA_OK) return s;
   if ((s = check_d_idx(d_idx)) != MSA_OK) return s;
+  if ((s = check_index_n(n, bk, k)) != MSA_OK) return s;
   if ((s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
       (s = check_ptr(block_ids, "block_ids")) != MSA_OK || (s = check_ptr(workspace, "workspace")) != MSA_OK)
     return s;
   const size_t need = index_ws_bytes(n, g, k);
   if (workspace_bytes < need)
     return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
-  return run_index_select(q_idx, k_idx, n, g, d_idx, k, block_ids, workspace, static_cast<cudaStream_t>(stream));
+  return run_index_select(q_idx, k_idx, n, g, d_idx, bk, k, block_ids, workspace, static_cast<cudaStream_t>(stream));
 }
 
 msa_status_t msa_index_select_static(const void* q_idx, const void* k_idx, int64_t n, int32_t g, int32_t d_idx,
@@ -941,8 +1161,12 @@ msa_status_t msa_index_select_static(const void* q_idx, const void* k_idx, int64
   if ((s = check_ptr(q_idx, "q_idx")) != MSA_OK || (s = check_ptr(k_idx, "k_idx")) != MSA_OK ||
       (s = check_ptr(block_ids, "block_ids")) != MSA_OK)
     return s;
-  // the launches are cut so that each fits the static scratch; the last query block alone
-  // needs 4 * g * 128 * (blocks - 1) bytes
+  if ((s = check_index_n(n, bk, k)) != MSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the one-kernel Index Branch keeps no block maxima in memory: no scratch at all
+  if (fused_index_ok(n, k)) return run_index_select(q_idx, k_idx, n, g, d_idx, bk, k, block_ids, nullptr, st);
+  // the two-kernel path: the launches are cut so that each fits the static scratch; the last
+  // query block alone needs 4 * g * 128 * (blocks - 1) bytes
   const int64_t nb = (n + 127) / 128;
   const size_t need = maxima_bytes(nb - 1, nb, g);
   if (need > kStaticScratchBytes)
@@ -956,7 +1180,6 @@ msa_status_t msa_index_select_static(const void* q_idx, const void* k_idx, int64
   L.maxima = static_cast<uint32_t*>(scratch);
   L.bytes = kStaticScratchBytes;
   L.cap = kStaticScratchBytes;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (d_idx) {
     case 32: return launch_index<32>(q_idx, k_idx, n, g, L, block_ids, k, st);
     case 64: return launch_index<64>(q_idx, k_idx, n, g, L, block_ids, k, st);
@@ -965,8 +1188,8 @@ msa_status_t msa_index_select_static(const void* q_idx, const void* k_idx, int64
 }
 
 size_t msa_sparse_attn_workspace(int64_t n, int32_t hq, int32_t g, int32_t d, int32_t bk, int32_t k) {
-  if (check_common(n, g, bk, k) != MSA_OK || check_main_dims(hq, g, d) != MSA_OK) return 0;
-  return attn_layout(nullptr, n, hq, g, d, k, 0).bytes;
+  if (check_common(n, g, bk, k) != MSA_OK || check_main_dims(hq, g, d) != MSA_OK || check_attn_n(n, bk) != MSA_OK) return 0;
+  return attn_layout(nullptr, n, hq, g, d, bk, k, 0).bytes;
 }
 
 msa_status_t msa_sparse_attn(const void* q, const void* k, const void* v, const int32_t* block_ids, int64_t n,
@@ -976,15 +1199,16 @@ msa_status_t msa_sparse_attn(const void* q, const void* k, const void* v, const 
   msa_status_t s;
   if ((s = check_common(n, g, bk, kk)) != MSA_OK) return s;
   if ((s = check_main_dims(hq, g, d)) != MSA_OK) return s;
+  if ((s = check_attn_n(n, bk)) != MSA_OK) return s;
   if (!(scale >= 0.0f) || std::isinf(scale)) return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if ((s = check_ptr(q, "q")) != MSA_OK || (s = check_ptr(k, "k")) != MSA_OK || (s = check_ptr(v, "v")) != MSA_OK ||
       (s = check_ptr(block_ids, "block_ids")) != MSA_OK || (s = check_ptr(o, "o")) != MSA_OK ||
       (s = check_ptr(workspace, "workspace")) != MSA_OK)
     return s;
-  const size_t need = attn_layout(nullptr, n, hq, g, d, kk, 0).bytes;
+  const size_t need = attn_layout(nullptr, n, hq, g, d, bk, kk, 0).bytes;
   if (workspace_bytes < need)
     return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
-  return run_sparse_attn(q, k, v, block_ids, n, hq, g, d, kk, scale, o, workspace, 0,
+  return run_sparse_attn(q, k, v, block_ids, n, hq, g, d, bk, kk, scale, o, workspace, 0,
                          static_cast<cudaStream_t>(stream));
 }
 
@@ -992,10 +1216,11 @@ size_t msa_forward_workspace(const msa_params* p) {
   if (!p) return 0;
   if (p->mode == MSA_MODE_PREFILL) {
     if (check_common(p->n, p->g, p->bk, p->k) != MSA_OK || check_main_dims(p->hq, p->g, p->d) != MSA_OK ||
-        check_d_idx(p->d_idx) != MSA_OK)
+        check_d_idx(p->d_idx) != MSA_OK || check_index_n(p->n, p->bk, p->k) != MSA_OK ||
+        check_attn_n(p->n, p->bk) != MSA_OK)
       return 0;
     if (p->query_chunk < 0 || p->query_chunk % 128 != 0) return 0;
-    const size_t a = attn_layout(nullptr, p->n, p->hq, p->g, p->d, p->k, p->query_chunk).bytes;
+    const size_t a = attn_layout(nullptr, p->n, p->hq, p->g, p->d, p->bk, p->k, p->query_chunk).bytes;
     const size_t b = index_ws_bytes(p->n, p->g, p->k);
     return prefill_ids_bytes(p->n, p->g, p->k) + std::max(a, b);
   }
@@ -1023,8 +1248,10 @@ msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, cons
       (s = check_ptr(o, "o")) != MSA_OK || (s = check_ptr(workspace, "workspace")) != MSA_OK)
     return s;
   if (block_ids_out && (s = check_ptr(block_ids_out, "block_ids_out")) != MSA_OK) return s;
+  if (p->lse_out && (s = check_ptr(p->lse_out, "lse_out")) != MSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (p->mode == MSA_MODE_PREFILL) {
+    if ((s = check_index_n(p->n, p->bk, p->k)) != MSA_OK || (s = check_attn_n(p->n, p->bk)) != MSA_OK) return s;
     if (p->query_chunk < 0 || p->query_chunk % 128 != 0)
       return fail(MSA_ERR_INVALID_ARG, "query_chunk=%lld must be a non-negative multiple of 128", (long long)p->query_chunk);
     const size_t need = msa_forward_workspace(p);
@@ -1033,8 +1260,9 @@ msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, cons
     uint8_t* w = static_cast<uint8_t*>(workspace);
     int32_t* ids = block_ids_out ? block_ids_out : reinterpret_cast<int32_t*>(w);
     void* rest = w + prefill_ids_bytes(p->n, p->g, p->k);
-    if ((s = run_index_select(q_idx, k_idx, p->n, p->g, p->d_idx, p->k, ids, rest, st)) != MSA_OK) return s;
-    return run_sparse_attn(q, k, v, ids, p->n, p->hq, p->g, p->d, p->k, p->scale, o, rest, p->query_chunk, st);
+    if ((s = run_index_select(q_idx, k_idx, p->n, p->g, p->d_idx, p->bk, p->k, ids, rest, st)) != MSA_OK) return s;
+    return run_sparse_attn(q, k, v, ids, p->n, p->hq, p->g, p->d, p->bk, p->k, p->scale, o, rest, p->query_chunk, st,
+                           nullptr, nullptr, p->lse_out);
   }
   if (p->mode == MSA_MODE_DECODE) {
     if (p->lmax < 1 || p->lmax > kMaxN) return fail(MSA_ERR_INVALID_ARG, "lmax=%lld out of range", (long long)p->lmax);
@@ -1084,10 +1312,12 @@ msa_status_t msa_forward_host(const msa_params* p, const void* q, const void* k,
   g_detail[0] = 0;
   if (!p) return fail(MSA_ERR_INVALID_ARG, "params is NULL");
   if (p->mode != MSA_MODE_PREFILL) return fail(MSA_ERR_UNSUPPORTED, "msa_forward_host takes prefill only");
+  if (p->lse_out) return fail(MSA_ERR_UNSUPPORTED, "msa_forward_host does not write lse_out (pass NULL)");
   msa_status_t s;
   if ((s = check_common(p->n, p->g, p->bk, p->k)) != MSA_OK) return s;
   if ((s = check_main_dims(p->hq, p->g, p->d)) != MSA_OK) return s;
   if ((s = check_d_idx(p->d_idx)) != MSA_OK) return s;
+  if ((s = check_index_n(p->n, p->bk, p->k)) != MSA_OK || (s = check_attn_n(p->n, p->bk)) != MSA_OK) return s;
   if (!(p->scale >= 0.0f) || std::isinf(p->scale)) return fail(MSA_ERR_INVALID_ARG, "scale must be finite and >= 0");
   if (p->query_chunk < 0 || p->query_chunk % 128 != 0)
     return fail(MSA_ERR_INVALID_ARG, "query_chunk=%lld must be a non-negative multiple of 128", (long long)p->query_chunk);
@@ -1103,8 +1333,8 @@ msa_status_t msa_forward_host(const msa_params* p, const void* q, const void* k,
   cudaStream_t cin = aux_stream(1), cout = aux_stream(2);
   if (cin == nullptr || cout == nullptr) return fail(MSA_ERR_CUDA, "could not create the copy streams");
   const int64_t n = p->n;
-  const AttnLayout L = attn_layout(nullptr, n, p->hq, p->g, p->d, p->k, p->query_chunk);
-  const int64_t rows_per_chunk = L.chunk_blocks * 128;
+  const AttnLayout L = attn_layout(nullptr, n, p->hq, p->g, p->d, p->bk, p->k, p->query_chunk);
+  const int64_t rows_per_chunk = L.chunk_tiles * 128;
   EventSet ev;   // 0 start, 1 index inputs in, 2 selection done, then per chunk: rows in, rows out
   if (!ev.make(size_t(3 + 2 * L.chunks))) return fail(MSA_ERR_CUDA, "cudaEventCreateWithFlags failed");
   const cudaEvent_t* chunk_in = ev.ev.data() + 3;
@@ -1139,14 +1369,14 @@ msa_status_t msa_forward_host(const msa_params* p, const void* q, const void* k,
   }
   int32_t* ids = reinterpret_cast<int32_t*>(H.ws);
   void* rest = static_cast<uint8_t*>(H.ws) + prefill_ids_bytes(n, p->g, p->k);
-  if ((s = run_index_select(H.qi, H.ki, n, p->g, p->d_idx, p->k, ids, rest, st)) != MSA_OK) return s;
+  if ((s = run_index_select(H.qi, H.ki, n, p->g, p->d_idx, p->bk, p->k, ids, rest, st)) != MSA_OK) return s;
   if (block_ids_out) {
     if (!cuda_ok(cudaEventRecord(ev.ev[2], st)) || !cuda_ok(cudaStreamWaitEvent(cout, ev.ev[2], 0)) ||
         !cuda_ok(cudaMemcpyAsync(block_ids_out, ids, size_t(n) * p->g * p->k * 4, cudaMemcpyDeviceToHost, cout)))
       return fail(MSA_ERR_CUDA, "block id copy failed");
   }
-  if ((s = run_sparse_attn(H.q, H.k, H.v, ids, n, p->hq, p->g, p->d, p->k, p->scale, H.o, rest, p->query_chunk, st,
-                           chunk_in, chunk_out)) != MSA_OK)
+  if ((s = run_sparse_attn(H.q, H.k, H.v, ids, n, p->hq, p->g, p->d, p->bk, p->k, p->scale, H.o, rest, p->query_chunk, st,
+                           chunk_in, chunk_out, nullptr)) != MSA_OK)
     return s;
   // each chunk's output rows go back as soon as its merge is done
   for (int64_t c = 0; c < L.chunks; ++c) {
@@ -1157,6 +1387,28 @@ msa_status_t msa_forward_host(const msa_params* p, const void* q, const void* k,
       return fail(MSA_ERR_CUDA, "output copy failed");
   }
   return MSA_OK;   // `stream` resumes once both copy streams are done (SideJoin)
+}
+
+size_t msa_index_kl_workspace(const msa_params* p) {
+  if (check_kl_params(p) != MSA_OK) return 0;
+  return attn_layout(nullptr, p->n, p->hq, p->g, p->d, p->bk, p->k, p->query_chunk, true).bytes;
+}
+
+msa_status_t msa_index_kl(const msa_params* p, const void* q, const void* k, const void* q_idx, const void* k_idx,
+                          const int32_t* block_ids, const float* lse, float idx_scale, float* kl, void* workspace,
+                          size_t workspace_bytes, void* stream) {
+  g_detail[0] = 0;
+  msa_status_t s;
+  if ((s = check_kl_params(p)) != MSA_OK) return s;
+  if (!(idx_scale >= 0.0f) || std::isinf(idx_scale)) return fail(MSA_ERR_INVALID_ARG, "idx_scale must be finite and >= 0");
+  if ((s = check_ptr(q, "q")) != MSA_OK || (s = check_ptr(k, "k")) != MSA_OK || (s = check_ptr(q_idx, "q_idx")) != MSA_OK ||
+      (s = check_ptr(k_idx, "k_idx")) != MSA_OK || (s = check_ptr(block_ids, "block_ids")) != MSA_OK ||
+      (s = check_ptr(lse, "lse")) != MSA_OK || (s = check_ptr(kl, "kl")) != MSA_OK ||
+      (s = check_ptr(workspace, "workspace")) != MSA_OK)
+    return s;
+  const size_t need = msa_index_kl_workspace(p);
+  if (workspace_bytes < need) return fail(MSA_ERR_WORKSPACE, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  return run_index_kl(p, q, k, q_idx, k_idx, block_ids, lse, idx_scale, kl, workspace, static_cast<cudaStream_t>(stream));
 }
 
 msa_status_t msa_profile_start(void) {
@@ -1200,6 +1452,14 @@ int32_t msa_profile_stop(msa_kernel_stat* out, int32_t max_out) {
     ++n;
   }
   return n;
+}
+
+msa_status_t msa_set_wait_limit_ns(uint64_t ns) {
+  g_detail[0] = 0;
+  const uint64_t v = (ns == 0) ? kWaitLimitNs : std::min<uint64_t>(ns, kWaitLimitNs);
+  cudaError_t e = cudaMemcpyToSymbol(msa::g_msa_wait_limit_ns, &v, sizeof(v));
+  if (e != cudaSuccess) return fail(MSA_ERR_CUDA, "set wait limit: %s", cudaGetErrorString(e));
+  return MSA_OK;
 }
 
 msa_status_t msa_get_device_error(void* stream) {

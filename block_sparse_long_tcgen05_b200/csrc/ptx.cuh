@@ -39,6 +39,19 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                "r"(bytes)
                : "memory");
 }
+// Non-blocking test of an mbarrier phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // try_wait with a suspend-time hint: the warp sleeps in hardware (up to the hint, in ns)
 // until the phase completes instead of spinning on issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
@@ -48,26 +61,55 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(static_cast<uint32_t>(kSuspendHintNs))
       : "memory");
   return ok != 0;
 }
 
-// Bounded wait on an mbarrier phase. Returns false when the wait gave up: after
-// kWaitLimitNs of wall time, or as soon as another role of the CTA raised *abort.
-// On a timeout it records MSA_ERR_TIMEOUT with the kernel id and sets *abort so the
-// other roles of the CTA stop too.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          int kernel_id) {
+// Per-CTA wait control in shared memory: the abort flag that one role raises for the others,
+// and the time limit of the waits that gate new work (loaded from g_msa_wait_limit_ns when
+// the kernel starts).
+struct WaitCtl {
+  volatile int abort;
+  int pad;
+  volatile uint64_t limit_ns;
+};
+
+__device__ __forceinline__ void wait_ctl_init(WaitCtl* ctl) {
+  ctl->abort = 0;
+  ctl->limit_ns = g_msa_wait_limit_ns;
+}
+
+// Bounded wait on an mbarrier phase. Returns false when the wait gave up: after the time
+// limit, or as soon as another role of the CTA raised ctl->abort. On a timeout it records
+// MSA_ERR_TIMEOUT with the kernel id and raises ctl->abort so the other roles stop too.
+// ctl == nullptr (the drains of work already in flight) waits up to kWaitLimitNs and never
+// stops early. Limits below the suspend hint poll without suspending, so that a short limit
+// is honoured.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* ctl, int kernel_id) {
+  uint64_t limit = static_cast<uint64_t>(kWaitLimitNs);
+  if (ctl != nullptr) limit = ctl->limit_ns;
+  if (limit < kSuspendHintNs) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+      if (mbar_test(bar, parity)) return true;
+      if (ctl != nullptr && ctl->abort) return false;
+      if (globaltimer_ns() - t0 > limit) {
+        record_error(MSA_ERR_TIMEOUT, kernel_id);
+        if (ctl != nullptr) ctl->abort = 1;
+        return false;
+      }
+    }
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (ctl != nullptr && ctl->abort) return false;
+      if (globaltimer_ns() - t0 > limit) {
         record_error(MSA_ERR_TIMEOUT, kernel_id);
-        if (abort != nullptr) *abort = 1;
+        if (ctl != nullptr) ctl->abort = 1;
         return false;
       }
     }
@@ -102,6 +144,15 @@ __device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, u
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// The same load with an L2 eviction-priority hint (a policy from createpolicy).
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1,
+                                                 int c2, int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
+}
 // TMA tensor store shared -> global (bulk-group completion).
 __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
                                              int c3) {
@@ -109,6 +160,15 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void*
                    reinterpret_cast<uint64_t>(map)),
                "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                : "memory");
+}
+// The same store with an L2 eviction-priority hint.
+__device__ __forceinline__ void tma_store_4d_hint(const CUtensorMap* map, const void* src, int c0, int c1, int c2,
+                                                  int c3, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4, %5}], [%1], %6;" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "l"(policy)
+      : "memory");
 }
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -212,19 +272,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// Non-blocking test of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // ----------------------------------------------------------------------------------
 // Descriptors
 // ----------------------------------------------------------------------------------
@@ -286,6 +333,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// L2 policy for data that is read again soon by other CTAs: evicted last.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
   return p;
 }
 

@@ -127,7 +127,7 @@ struct TopkDecodeParams {
   const uint32_t* maxima;   // [B, G, nbmax]
   int32_t* block_ids;       // [B, G, k]
   const int32_t* seqlens;
-  int B, G, k, nbmax;
+  int B, G, k, nbmax, bk;
 };
 
 }  // namespace msa

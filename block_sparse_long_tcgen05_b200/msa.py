@@ -23,7 +23,8 @@ MODE_PREFILL, MODE_DECODE = 0, 1
 EXPORTS = ("msa_index_select_workspace", "msa_index_select", "msa_sparse_attn_workspace", "msa_sparse_attn",
            "msa_forward_workspace", "msa_forward", "msa_get_device_error", "msa_status_string",
            "msa_last_error_detail", "msa_profile_start", "msa_profile_stop", "msa_index_select_static",
-           "msa_forward_host_device_bytes", "msa_forward_host")
+           "msa_forward_host_device_bytes", "msa_forward_host", "msa_index_kl_workspace", "msa_index_kl",
+           "msa_set_wait_limit_ns")
 
 
 class MsaError(RuntimeError):
@@ -36,7 +37,8 @@ class MsaParams(ctypes.Structure):
     _fields_ = [("mode", ctypes.c_int32), ("hq", ctypes.c_int32), ("g", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("d_idx", ctypes.c_int32), ("bk", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("scale", ctypes.c_float), ("n", ctypes.c_int64),
-                ("lmax", ctypes.c_int64), ("seqlens", ctypes.c_void_p), ("query_chunk", ctypes.c_int64)]
+                ("lmax", ctypes.c_int64), ("seqlens", ctypes.c_void_p), ("query_chunk", ctypes.c_int64),
+                ("lse_out", ctypes.c_void_p)]
 
 
 class MsaKernelStat(ctypes.Structure):
@@ -72,6 +74,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
         "msa_index_select_static": (c_i32, [c_p, c_p, c_i64, c_i32, c_i32, c_i32, c_i32, c_p, c_p]),
         "msa_forward_host_device_bytes": (c_sz, [pp]),
         "msa_forward_host": (c_i32, [pp, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_p, c_sz, c_p]),
+        "msa_index_kl_workspace": (c_sz, [pp]),
+        "msa_index_kl": (c_i32, [pp, c_p, c_p, c_p, c_p, c_p, c_p, c_f, c_p, c_p, c_sz, c_p]),
+        "msa_set_wait_limit_ns": (c_i32, [ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -224,11 +229,41 @@ def forward_host(p: MsaParams, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
 
 def prefill(q, k, v, q_idx, k_idx, topk: int, bk: int = 128, scale: float = 0.0, query_chunk: int = 0,
             block_ids: torch.Tensor | None = None, o: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None) -> torch.Tensor:
+            workspace: torch.Tensor | None = None, lse: torch.Tensor | None = None) -> torch.Tensor:
+    """Both branches of one sequence; with `lse` (float32 [N, Hq]) also the log-sum-exp of
+    every (query, head)'s logits over its selected tokens, as index_kl takes it."""
     N, Hq, d = q.shape
     G, d_idx = q_idx.shape[1], q_idx.shape[2]
     p = prefill_params(N, Hq, G, d, d_idx, topk, bk, scale, query_chunk)
+    if lse is not None:
+        if lse.dtype != torch.float32 or tuple(lse.shape) != (N, Hq):
+            raise ValueError("lse must be float32 [N, Hq]")
+        p.lse_out = _ptr(lse)
     return msa_forward(p, q, k, v, q_idx, k_idx, o=o, block_ids=block_ids, workspace=workspace)
+
+
+def index_kl(q, k, q_idx, k_idx, block_ids: torch.Tensor, lse: torch.Tensor, bk: int = 128, scale: float = 0.0,
+             idx_scale: float = 0.0, query_chunk: int = 0, kl: torch.Tensor | None = None,
+             workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Index-branch KL loss forward (msa_index_kl): KL(P_main || P_idx) per (query, group) ->
+    float32 [N, G]; block_ids and lse as the prefill forward produced them."""
+    lib = load_library()
+    N, Hq, d = q.shape
+    G, d_idx = q_idx.shape[1], q_idx.shape[2]
+    topk = block_ids.shape[2]
+    if block_ids.dtype != torch.int32 or lse.dtype != torch.float32:
+        raise ValueError("block_ids must be int32 and lse float32")
+    p = prefill_params(N, Hq, G, d, d_idx, topk, bk, scale, query_chunk)
+    if kl is None:
+        kl = torch.empty(N, G, dtype=torch.float32, device=q.device)
+    need = lib.msa_index_kl_workspace(ctypes.byref(p))
+    if need == 0:
+        raise MsaError(2, "unsupported shape for msa_index_kl")
+    ws = _workspace(need, q.device, workspace)
+    _check(lib.msa_index_kl(ctypes.byref(p), _bf16(q, "q"), _bf16(k, "k"), _bf16(q_idx, "q_idx"),
+                            _bf16(k_idx, "k_idx"), _ptr(block_ids), _ptr(lse), idx_scale, _ptr(kl), _ptr(ws),
+                            ws.numel(), _stream(q.device)))
+    return kl
 
 
 def decode(q, k_cache, v_cache, q_idx, k_idx_cache, seqlens, topk: int, bk: int = 128, scale: float = 0.0,
@@ -255,6 +290,11 @@ def check_device_error(device=None) -> None:
     st = msa_get_device_error(device)
     if st != MSA_OK:
         raise MsaError(st, load_library().msa_last_error_detail().decode())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Time limit of the kernels' gating waits on the current device (0: the 2 s default)."""
+    _check(load_library().msa_set_wait_limit_ns(int(ns)))
 
 
 def msa_profile_start() -> None:

@@ -191,6 +191,27 @@ def attend_rows(q, k, v, block_ids: np.ndarray, rows, Bk: int, scale: float | No
     return out
 
 
+def lse_rows(q, k, block_ids: np.ndarray, rows, Bk: int, scale: float | None = None) -> np.ndarray:
+    """Natural-log log-sum-exp of each (row, head)'s scaled logits over the tokens of its
+    group's selected blocks (j <= i): the normaliser of step 4's softmax. [r, Hq] fp64."""
+    rows = np.asarray(list(rows), dtype=np.int64)
+    N, Hq, d = q.shape
+    G = k.shape[1]
+    R = Hq // G
+    scale = (1.0 / np.sqrt(d)) if not scale else scale
+    out = np.zeros((len(rows), Hq), dtype=np.float64)
+    for t, i in enumerate(rows):
+        i = int(i)
+        qi = to_f64(q[i])
+        for g in range(G):
+            toks = selected_tokens(block_ids[t, g], i, Bk)
+            tk = torch.as_tensor(toks) if isinstance(k, torch.Tensor) else toks
+            logits = (to_f64(k[tk, g, :]) @ qi[g * R:(g + 1) * R].T).T * scale    # [R, T]
+            m = logits.max(axis=1)
+            out[t, g * R:(g + 1) * R] = m + np.log(np.exp(logits - m[:, None]).sum(axis=1))
+    return out
+
+
 def prefill_rows(inp: dict, rows, Bk: int, k: int, scale: float | None = None):
     """Both branches for sampled query rows of one prefill sequence.
 

@@ -53,7 +53,11 @@ def test_validation_rejects_bad_arguments_without_cuda(lib):
     # misaligned pointer
     assert lib.msa_index_select(P + 2, P, 256, 2, 32, 128, 4, P, P, 1 << 30, None) == 1
     # unsupported block size, d_idx, k
-    assert lib.msa_index_select(P, P, 256, 2, 32, 64, 4, P, P, 1 << 30, None) == 2
+    assert lib.msa_index_select(P, P, 256, 2, 32, 96, 4, P, P, 1 << 30, None) == 2
+    # block sizes below 128 take the one-kernel Index Branch only (k in 4, 8, 16, 32)
+    assert lib.msa_index_select(P, P, 256, 2, 32, 64, 5, P, P, 1 << 30, None) == 2
+    assert lib.msa_index_select_workspace(256, 2, 32, 64, 5) == 0
+    assert lib.msa_index_select_workspace(256, 2, 32, 32, 8) > 0
     assert lib.msa_index_select(P, P, 256, 2, 48, 128, 4, P, P, 1 << 30, None) == 2
     assert lib.msa_index_select(P, P, 256, 2, 32, 128, 33, P, P, 1 << 30, None) == 2
     # bad n
@@ -115,5 +119,35 @@ def test_workspace_sizes_grow_with_problem(lib):
     assert 0 < lib.msa_index_select_workspace(131072, 8, 128, 128, 16) <= 4096
     # k = 5 takes the two-kernel path: the packed maxima triangle lives in the workspace
     assert lib.msa_index_select_workspace(131072, 8, 128, 128, 5) >= 4 * 8 * 128 * (1024 * 1023 // 2)
-    # beyond 256K tokens the two-kernel path is used for every k
-    assert lib.msa_index_select_workspace(524288, 8, 128, 128, 16) >= 4 * 8 * 128 * (4096 * 4095 // 2) // 8
+    # the one-kernel path serves k = 16 at every length (1M tokens: no maxima either)
+    assert 0 < lib.msa_index_select_workspace(1 << 20, 8, 128, 128, 16) <= 4096
+    assert lib.msa_index_select_workspace(524288, 8, 128, 128, 12) >= 4 * 8 * 128 * (4096 * 4095 // 2) // 8
+
+
+def test_sequence_length_limits_are_checked_before_any_launch(lib):
+    """Each path's longest sequence is validated with the other arguments, so nothing is
+    enqueued for a problem that would fail part-way: the two-kernel Index Branch (odd k, or
+    long sequences) takes at most 32768 query blocks (its key-run table), the Main Branch at
+    most 14528 blocks (the CSR build's shared-memory masks)."""
+    P = 1 << 12
+    two_kernel_max = 32768 * 128
+    csr_max = 14528 * 128
+    # just above the two-kernel limit (g = 1): refused, and so is its workspace query
+    assert lib.msa_index_select_workspace(two_kernel_max + 1, 1, 32, 128, 5) == 0
+    assert lib.msa_index_select(P, P, two_kernel_max + 1, 1, 32, 128, 5, P, P, 1 << 40, None) == 2
+    assert b"two-kernel" in lib.msa_last_error_detail()
+    assert lib.msa_index_select_static(P, P, 5_000_000, 1, 32, 128, 5, P, None) == 2
+    assert b"two-kernel" in lib.msa_last_error_detail()
+    # at the limit the workspace query still answers
+    assert lib.msa_index_select_workspace(two_kernel_max, 1, 32, 128, 5) > 0
+    # Main Branch: the limit counts blocks, so it is 4x shorter in tokens at bk = 32
+    assert lib.msa_sparse_attn_workspace(14528 * 32, 8, 2, 64, 32, 4) > 0
+    assert lib.msa_sparse_attn_workspace(14528 * 32 + 1, 8, 2, 64, 32, 4) == 0
+    assert lib.msa_sparse_attn_workspace(csr_max, 8, 2, 64, 128, 4) > 0
+    assert lib.msa_sparse_attn_workspace(csr_max + 1, 8, 2, 64, 128, 4) == 0
+    assert lib.msa_sparse_attn(P, P, P, P, csr_max + 1, 8, 2, 64, 128, 4, 0.0, P, P, 1 << 40, None) == 2
+    assert b"Main Branch" in lib.msa_last_error_detail()
+    p = msa.prefill_params(csr_max + 1, 8, 2, 64, 32, 4)
+    assert lib.msa_forward_workspace(ctypes.byref(p)) == 0
+    assert lib.msa_forward(ctypes.byref(p), P, P, P, P, P, None, P, P, 1 << 40, None) == 2
+    assert lib.msa_forward_host(ctypes.byref(p), P, P, P, P, P, None, P, P, 1 << 40, None) == 2

@@ -27,6 +27,19 @@ def assert_close(o_gpu, o_ref, what=""):
                            f"max err {err.max():.3e}, worst excess {(err - bound).max():.3e}")
 
 
+def host_f64(inp: dict) -> dict:
+    """fp64 numpy copies of the inputs (exact): the oracle then indexes plain arrays, which
+    is much faster than converting torch slices row by row."""
+    return {n: t.detach().cpu().double().numpy() if t.is_floating_point() else t.detach().cpu().numpy()
+            for n, t in inp.items()}
+
+
+def oracle_prefill(inp: dict, rows, Bk: int, k: int):
+    h = host_f64(inp)
+    ids, _ = orc.index_select_rows(h["q_idx"], h["k_idx"], rows, Bk, k)
+    return ids, orc.attend_rows(h["q"], h["k"], h["v"], ids, rows, Bk)
+
+
 def sample_rows(N, k, Bk=128, n=64, seed=0):
     must = [0, Bk - 1, Bk, k * Bk - 1, k * Bk, N - 1]
     rng = np.random.default_rng(seed)
@@ -34,16 +47,16 @@ def sample_rows(N, k, Bk=128, n=64, seed=0):
     return sorted(set(x for x in must + extra if 0 <= x < N))
 
 
-def cfg_of(N, Hq, G, d, d_idx, k, hot=0.0, seed=77, idx_range=4):
+def cfg_of(N, Hq, G, d, d_idx, k, hot=0.0, seed=77, idx_range=4, Bk=128):
     return synth.PrefillConfig("t", N=N, Hq=Hq, G=G, d=d, d_idx=d_idx, k=k, idx_range=idx_range,
-                               hot_frac=hot, seed=seed)
+                               hot_frac=hot, seed=seed, Bk=Bk)
 
 
 def check_prefill(cfg, rows=None, query_chunk=0, check_all_ids=True):
     dev = torch.device("cuda")
     inp = synth.prefill_inputs(cfg, device=dev)
     ids_gpu = torch.empty(cfg.N, cfg.G, cfg.k, dtype=torch.int32, device=dev)
-    o = msa.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cfg.k, block_ids=ids_gpu,
+    o = msa.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cfg.k, bk=cfg.Bk, block_ids=ids_gpu,
                     query_chunk=query_chunk)
     msa.check_device_error()
     if rows is None:
@@ -54,7 +67,7 @@ def check_prefill(cfg, rows=None, query_chunk=0, check_all_ids=True):
         ids_ref, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, cfg.Bk, cfg.k)
         o_ref = orc.attend_rows(inp["q"], inp["k"], inp["v"], ids_ref, rows, cfg.Bk)
     else:
-        ids_ref, o_ref = orc.prefill_rows(inp, rows, cfg.Bk, cfg.k)
+        ids_ref, o_ref = oracle_prefill(inp, rows, cfg.Bk, cfg.k)
     ids_g = ids_gpu.cpu().numpy()
     np.testing.assert_array_equal(ids_g[rows], ids_ref)
     if check_all_ids:
@@ -88,7 +101,22 @@ def test_index_select_all_rows_bit_exact(cuda_ok, N, G, d_idx, k):
     inp = synth.prefill_inputs(cfg, device="cuda")
     ids = msa.msa_index_select(inp["q_idx"], inp["k_idx"], k)
     msa.check_device_error()
-    ref, _ = orc.index_select_rows(inp["q_idx"].cpu(), inp["k_idx"].cpu(), range(N), 128, k)
+    h = host_f64(inp)
+    ref, _ = orc.index_select_rows(h["q_idx"], h["k_idx"], range(N), 128, k)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("N,G,d_idx,k,Bk", [(2048 + 77, 2, 128, 16, 64), (3000, 3, 32, 8, 32),
+                                             (5000, 2, 64, 32, 32), (4000, 8, 128, 4, 64), (700, 1, 32, 16, 32)])
+def test_index_select_block_sizes_bit_exact(cuda_ok, N, G, d_idx, k, Bk):
+    """Block sizes 64 and 32 of the block-size ablation (hyper.ai page, Experiment): each
+    128-key tile holds several blocks, and rows see the earlier blocks of their own tile."""
+    cfg = cfg_of(N, G, G, 64, d_idx, k, hot=0.05, idx_range=3, Bk=Bk)
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    ids = msa.msa_index_select(inp["q_idx"], inp["k_idx"], k, bk=Bk)
+    msa.check_device_error()
+    h = host_f64(inp)
+    ref, _ = orc.index_select_rows(h["q_idx"], h["k_idx"], range(N), Bk, k)
     np.testing.assert_array_equal(ids.cpu().numpy(), ref)
 
 
@@ -126,11 +154,12 @@ def test_index_select_negative_zero_ties(cuda_ok):
 def test_sparse_attn_all_rows(cuda_ok, N, Hq, G, d):
     cfg = cfg_of(N, Hq, G, d, 32, 4, seed=5)
     inp = synth.prefill_inputs(cfg, device="cuda")
-    ref_ids, _ = orc.index_select_rows(inp["q_idx"].cpu(), inp["k_idx"].cpu(), range(N), 128, 4)
+    h = host_f64(inp)
+    ref_ids, _ = orc.index_select_rows(h["q_idx"], h["k_idx"], range(N), 128, 4)
     ids = torch.from_numpy(ref_ids).cuda()
     o = msa.msa_sparse_attn(inp["q"], inp["k"], inp["v"], ids)
     msa.check_device_error()
-    o_ref = orc.attend_rows(inp["q"].cpu(), inp["k"].cpu(), inp["v"].cpu(), ref_ids, range(N), 128)
+    o_ref = orc.attend_rows(h["q"], h["k"], h["v"], ref_ids, range(N), 128)
     assert_close(o.float().cpu().numpy(), o_ref, "sparse_attn")
 
 
@@ -163,6 +192,27 @@ def test_forward_dense_reduction(cuda_ok):
 def test_forward_query_chunks(cuda_ok, query_chunk):
     cfg = cfg_of(1300, 16, 2, 128, 64, 4, hot=0.1)
     check_prefill(cfg, query_chunk=query_chunk)
+
+
+@pytest.mark.parametrize("N,Hq,G,d,d_idx,k,rows", [(4000, 16, 2, 128, 128, 17, None), (5000, 16, 2, 128, 128, 32, None),
+                                                    (4600 + 33, 16, 4, 64, 64, 32, None),
+                                                    (5000, 64, 8, 128, 128, 32, 400)])
+def test_forward_large_k(cuda_ok, N, Hq, G, d, d_idx, k, rows):
+    """k above 16: slot ids 16..31 in the inverted index, the merge's combination of more than
+    16 slots, and (k = 32) the one-kernel Index Branch's longest running list; k = 17 takes
+    the two-kernel Index Branch. R = 8 heads per group with hot blocks; every row (or, at
+    the workload's 64 heads, seeded rows plus the edge rows); the sequences are long enough
+    (more than k blocks) that the later rows make a real selection."""
+    cfg = cfg_of(N, Hq, G, d, d_idx, k, hot=0.05, seed=40 + k)
+    check_prefill(cfg, rows=None if rows is None else sample_rows(N, k, n=rows, seed=k))
+
+
+@pytest.mark.parametrize("N,Hq,G,d,d_idx,k,Bk", [(3000, 16, 2, 128, 128, 16, 64), (2500, 8, 2, 64, 32, 8, 32),
+                                                 (2000 + 33, 64, 8, 128, 128, 32, 32), (1500, 4, 4, 64, 64, 4, 64)])
+def test_forward_block_sizes_all_rows(cuda_ok, N, Hq, G, d, d_idx, k, Bk):
+    """Both branches at block sizes 64 and 32: K/V blocks of Bk keys in the KV-outer pass, the
+    causal mask inside Bk-token local blocks, Bk-block buckets in the inverted index."""
+    check_prefill(cfg_of(N, Hq, G, d, d_idx, k, hot=0.05, seed=60 + Bk + k, Bk=Bk), query_chunk=1024)
 
 
 def test_forward_32k_sampled(cuda_ok):
@@ -202,7 +252,7 @@ def test_forward_host_matches_device_path(cuda_ok):
         assert torch.equal(ids_h, ids_d.cpu())
         assert torch.equal(o_h, o_d.cpu())
     rows = sample_rows(cfg.N, cfg.k, n=24, seed=5)
-    ids_ref, o_ref = orc.prefill_rows(inp, rows, cfg.Bk, cfg.k)
+    ids_ref, o_ref = oracle_prefill(inp, rows, cfg.Bk, cfg.k)
     np.testing.assert_array_equal(ids_h.numpy()[rows], ids_ref)
     assert_close(o_h.float().numpy()[rows], o_ref, "forward_host o")
 
@@ -225,6 +275,11 @@ def test_group_shard_equals_slice_of_full_forward(cuda_ok):
         msa.check_device_error()
         assert torch.equal(ids_p, ids_full[:, gs])
         assert torch.equal(o_p, o_full[:, hs])
+        # and against the oracle on the rank's own inputs: its groups of the full problem
+        rows = sample_rows(cfg.N, cfg.k, n=24, seed=40 + r)
+        ids_ref, o_ref = oracle_prefill(inp, rows, cfg.Bk, cfg.k)
+        np.testing.assert_array_equal(ids_p.cpu().numpy()[rows], ids_ref[:, gs])
+        assert_close(o_p.float().cpu().numpy()[rows], o_ref[:, hs], f"group shard {r}")
 
 
 # ---------------------------------------------------------------- decode
@@ -233,7 +288,7 @@ def check_decode(cfg, lengths, seqs=None, Lmax=None):
     inp = synth.decode_inputs(cfg, device="cuda", lengths=lengths, Lmax=Lmax)
     ids = torch.empty(len(lengths), cfg.G, cfg.k, dtype=torch.int32, device="cuda")
     o = msa.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["q_idx"], inp["k_idx_cache"], inp["seqlens"],
-                   cfg.k, block_ids=ids)
+                   cfg.k, bk=cfg.Bk, block_ids=ids)
     msa.check_device_error()
     seqs = list(range(len(lengths))) if seqs is None else seqs
     ids_ref, o_ref = orc.decode_rows(inp, seqs, cfg.Bk, cfg.k)
@@ -246,6 +301,22 @@ def test_decode_varied_lengths(cuda_ok):
     check_decode(cfg, [1, 2, 127, 128, 129, 2048, 2049, 5000, 9000], Lmax=9001)
 
 
+@pytest.mark.parametrize("k", [17, 32])
+def test_decode_large_k(cuda_ok, k):
+    """k above 16 on the decode path (its merge combines the slots past the first 16 one by
+    one); lengths on both sides of k blocks and with every kind of partial last block."""
+    cfg = synth.DecodeConfig("t", B=6, L=0, Hq=64, G=8, d=128, d_idx=128, k=k, hot_frac=0.05, seed=11 + k)
+    check_decode(cfg, [k * 128 - 1, k * 128, k * 128 + 1, 5000, 9000, 300], Lmax=9001)
+
+
+@pytest.mark.parametrize("Bk,k", [(64, 16), (32, 8)])
+def test_decode_block_sizes(cuda_ok, Bk, k):
+    """Decode at block sizes 64 and 32: a scan CTA covers several blocks of 128 tokens, the
+    local block is the last partial Bk-block."""
+    cfg = synth.DecodeConfig("t", B=7, L=0, Hq=64, G=8, d=128, d_idx=128, k=k, Bk=Bk, hot_frac=0.05, seed=13 + Bk)
+    check_decode(cfg, [1, Bk - 1, Bk, Bk + 1, k * Bk + 3, 3000, 5001], Lmax=5001)
+
+
 def test_decode_small_dims(cuda_ok):
     cfg = synth.DecodeConfig("t", B=5, L=0, Hq=8, G=2, d=64, d_idx=32, k=4, hot_frac=0.0, seed=10, idx_range=3)
     check_decode(cfg, [300, 700, 128, 1, 4096])
@@ -255,3 +326,25 @@ def test_decode_small_dims(cuda_ok):
 def test_decode_full_size_sampled(cuda_ok):
     """Batch 64 x 131073 tokens (the decode configuration); the oracle checks 6 sequences."""
     check_decode(synth.DEC128K, [131073] * 64, seqs=[0, 1, 17, 31, 48, 63])
+
+
+# ---------------------------------------------------------------- failure detection
+
+def test_wait_timeout_is_reported_and_the_device_stays_usable(cuda_ok):
+    """A gating-wait limit of 1 ns makes every pipelined kernel give up at its first wait that
+    is not already satisfied: the call reports MSA_ERR_TIMEOUT through the error word (no hang,
+    no fault: work already in flight is drained with the normal limit). With the default limit
+    restored, the same device computes the tiny configuration exactly as before."""
+    cfg = synth.TINY
+    inp = synth.prefill_inputs(cfg, device="cuda")
+    torch.cuda.synchronize()
+    msa.set_wait_limit_ns(1)
+    try:
+        msa.prefill(inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"], cfg.k)
+        st = msa.msa_get_device_error()
+    finally:
+        torch.cuda.synchronize()
+        msa.set_wait_limit_ns(0)
+    assert st == 5, msa.STATUS.get(st)
+    assert msa.msa_get_device_error() == 0   # cleared
+    check_prefill(cfg)

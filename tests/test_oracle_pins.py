@@ -412,3 +412,23 @@ def test_kl_nonnegative_and_zero_on_the_first_row():
     kl = orc.index_kl_rows(inp["q"], inp["k"], inp["q_idx"], inp["k_idx"], ids, rows, 128)
     assert kl.min() > -1e-12
     assert np.abs(kl[-1]).max() < 1e-15
+
+
+def test_lse_rows_closed_forms():
+    """The Main Branch's log-sum-exp: row 0 sees one token, so lse = scale q0.k0; and exp(lse)
+    is the softmax normaliser: sum_j exp(l_j - lse) = 1 over the selected tokens (checked
+    with torch.logsumexp on the same logits)."""
+    cfg, inp = _kl_inputs(N=400, Hq=4, G=2, d=32, d_idx=16, seed=17, k=2)
+    rows = [0, 77, 260, 399]
+    ids, _ = orc.index_select_rows(inp["q_idx"], inp["k_idx"], rows, 128, cfg.k)
+    lse = orc.lse_rows(inp["q"], inp["k"], ids, rows, 128)
+    q = inp["q"].double()
+    k = inp["k"].double()
+    for h in range(4):
+        assert lse[0, h] == pytest.approx(float(q[0, h] @ k[0, h // 2]) / math.sqrt(32), rel=1e-13)
+    for t, i in enumerate(rows):
+        for h in range(4):
+            g = h // 2
+            toks = [j for b in ids[t, g] if b >= 0 for j in range(b * 128, min(b * 128 + 128, i + 1))]
+            want = torch.logsumexp(k[toks, g] @ q[i, h] / math.sqrt(32), dim=0).item()
+            assert lse[t, h] == pytest.approx(want, rel=1e-12)
