@@ -258,20 +258,30 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_after();
         if (tile_present && kb < qb + kDiag) {
           const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + ab * 256 + tile * 128;
-          // the whole 128-column row in one TMEM round trip, then independent max chains
+          // the 128-column row in two halves: the first half's max chains run while the second
+          // half is in flight, then the accumulator is handed back
           uint32_t v[4][32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) tmem_ld32(taddr + c * 32, v[c]);
+          tmem_ld32(taddr, v[0]);
+          tmem_ld32(taddr + 32, v[1]);
           tmem_ld_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acc_empty[ab]);
+          tmem_ld32(taddr + 64, v[2]);
+          tmem_ld32(taddr + 96, v[3]);
           if constexpr (F == 1) {
             float m8[8];
 #pragma unroll
             for (int j = 0; j < 8; ++j) m8[j] = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int j = 0; j < 32; j += 2)
+                m8[(c * 16 + (j >> 1)) & 7] =
+                    max3f(m8[(c * 16 + (j >> 1)) & 7], __uint_as_float(v[c][j]), __uint_as_float(v[c][j + 1]));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
+#pragma unroll
+            for (int c = 2; c < 4; ++c)
 #pragma unroll
               for (int j = 0; j < 32; j += 2)
                 m8[(c * 16 + (j >> 1)) & 7] =
@@ -279,6 +289,10 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             offer(fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))),
                   kb, true);
           } else {
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[ab]);
             constexpr int CPS = BK / 32;     // 32-column chunks per block
 #pragma unroll
             for (int f = 0; f < F; ++f) {

@@ -87,6 +87,7 @@ __device__ __forceinline__ void wait_ctl_init(WaitCtl* ctl) {
 // stops early. Limits below the suspend hint poll without suspending, so that a short limit
 // is honoured.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, WaitCtl* ctl, int kernel_id) {
+  if (mbar_test(bar, parity)) return true;   // already complete: nothing else to read
   uint64_t limit = static_cast<uint64_t>(kWaitLimitNs);
   if (ctl != nullptr) limit = ctl->limit_ns;
   if (limit < kSuspendHintNs) {
