@@ -626,6 +626,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--headline-only", action="store_true",
                     help="skip the report of the other synthetic configurations (N = 1)")
+    ap.add_argument("--only-kl", action="store_true",
+                    help="measure only the index-branch KL loss forward on --workload (for profiling)")
     ap.add_argument("--shard", choices=["sequences", "groups"], default="sequences",
                     help="N > 1: one independent sequence per GPU (weak scaling) or the GQA groups of one "
                          "sequence split over the GPUs (strong scaling); no collective either way")
@@ -646,6 +648,15 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
+        elif args.only_kl:
+            from block_sparse_long_tcgen05_b200 import msa
+            msa.load_library()
+            dev = torch.device("cuda", local)
+            torch.cuda.set_device(dev)
+            peaks, _ = load_peaks()
+            out = kl_report(synth.CONFIGS[args.workload], dev, torch.cuda.current_stream(dev), args, peaks)
+            if rank == 0:
+                print(json.dumps({"index_kl": out}), flush=True)
         else:
             run_ours(args, world, rank, local)
     finally:

@@ -225,16 +225,18 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       int Lb[KM];
 #pragma unroll
       for (int p = 0; p < KM; ++p) { Ls[p] = 0u; Lb[p] = -1; }
-      // Blocks that beat the list's current last entry wait in a 4-entry buffer (ascending
-      // block order) and go into the list together when some row of the warp has 4: the
+      // Blocks that beat the list's current last entry wait in a CB-entry buffer (ascending
+      // block order) and go into the list together when some row of the warp has CB: the
       // insertion network, which the whole warp runs whenever any row needs it, then runs
-      // about as often as the busiest row has candidates instead of whenever any row has one.
-      uint32_t cu[4];
-      int cb[4];
+      // about as often as the busiest row has candidates instead of whenever any row has one
+      // (measured: 8 and 16 entries are slower than 4).
+      constexpr int CB = 4;
+      uint32_t cu[CB];
+      int cb[CB];
       int nc = 0;
       auto flush = [&]() {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < CB; ++c)
           if (c < nc) topk_insert_ascending<KM>(Ls, Lb, cu[c], cb[c]);
         nc = 0;
       };
@@ -245,11 +247,11 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
         if (valid && u > Ls[KM - 1]) {
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < CB; ++c)
             if (nc == c) { cu[c] = u; cb[c] = b; }
           ++nc;
         }
-        if (__any_sync(0xffffffffu, nc == 4)) flush();
+        if (__any_sync(0xffffffffu, nc == CB)) flush();
       };
       for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
         const int ab = static_cast<int>(ik & 1);

@@ -144,7 +144,9 @@ struct MergeStreamLayout {
 __device__ __forceinline__ float bf16lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
-template <int D>
+// kLse: also write each (query, head)'s log-sum-exp (a separate instantiation, so the common
+// path carries no code for it).
+template <int D, bool kLse>
 __global__ void __launch_bounds__(kMergeThreads, 1)
 merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant__ MergeStreamLayout S) {
   extern __shared__ uint8_t smem_raw[];
@@ -221,9 +223,7 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
       float* wt = reinterpret_cast<float*>(st + S.w_off);
       // valid ids come first (ascending, -1 padded); k <= 32, one lane per slot
       const int nv = __popc(__ballot_sync(0xffffffffu, lane < P.k && ids[lane] >= 0));
-      const int64_t i = P.row0 + u / P.G;
-      const int g = static_cast<int>(u % P.G);
-      float* lse_row = (P.lse != nullptr && lane == 0) ? P.lse + i * Hq + g * P.R : nullptr;
+
       // ---- weights of the heads this warp combines (32 is a multiple of CPR, so each head's
       // tasks belong to one warp and no other warp reads its weights)
       for (int t0 = gw * 32; t0 < tasks; t0 += kMergeGroupThreads) {
@@ -238,11 +238,14 @@ merge_stream_kernel(const __grid_constant__ MergeParams P, const __grid_constant
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
           if (lane < P.k) wt[lane * P.R + r] = (W > 0.0f) ? __fdividef(e, W) : 0.0f;
-          if (lse_row != nullptr)   // logits are in log2 units: scale back by ln 2
-            lse_row[r] = (M + __log2f(W)) * 0.6931471805599453f;
+          if constexpr (kLse) {   // logits are in log2 units: scale back by ln 2
+            if (lane == 0) P.lse[(P.row0 + u / P.G) * Hq + (u % P.G) * P.R + r] = (M + __log2f(W)) * 0.6931471805599453f;
+          }
         }
       }
       __syncwarp();
+      const int64_t i = P.row0 + u / P.G;
+      const int g = static_cast<int>(u % P.G);
       // ---- combine: thread task (r, c) = head r, 16-byte chunk c of its D-wide row
       for (int task = gt; task < tasks; task += kMergeGroupThreads) {
         const int r = task / CPR, c = task % CPR;

@@ -649,16 +649,24 @@ msa_status_t launch_merge_stream(const MergeParams& mp, int d, int max_grid, cud
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
   std::call_once(once, [] {
-    attr = set_smem(merge_stream_kernel<128>, 227 * 1024);
-    if (attr == MSA_OK) attr = set_smem(merge_stream_kernel<64>, 227 * 1024);
+    attr = set_smem(merge_stream_kernel<128, false>, 227 * 1024);
+    if (attr == MSA_OK) attr = set_smem(merge_stream_kernel<64, false>, 227 * 1024);
+    if (attr == MSA_OK) attr = set_smem(merge_stream_kernel<128, true>, 227 * 1024);
+    if (attr == MSA_OK) attr = set_smem(merge_stream_kernel<64, true>, 227 * 1024);
   });
   if (attr != MSA_OK) return attr;
   const int64_t units = mp.rows * mp.G;
   const int grid = int(std::min<int64_t>(max_grid, units));
   {
     ProfScope ps(kPMerge, st);
-    if (d == 128) merge_stream_kernel<128><<<grid, kMergeThreads, smem, st>>>(mp, L);
-    else merge_stream_kernel<64><<<grid, kMergeThreads, smem, st>>>(mp, L);
+    const bool lse = mp.lse != nullptr;
+    if (d == 128) {
+      if (lse) merge_stream_kernel<128, true><<<grid, kMergeThreads, smem, st>>>(mp, L);
+      else merge_stream_kernel<128, false><<<grid, kMergeThreads, smem, st>>>(mp, L);
+    } else {
+      if (lse) merge_stream_kernel<64, true><<<grid, kMergeThreads, smem, st>>>(mp, L);
+      else merge_stream_kernel<64, false><<<grid, kMergeThreads, smem, st>>>(mp, L);
+    }
   }
   MSA_CHECK_LAUNCH();
   return MSA_OK;
@@ -1265,6 +1273,7 @@ msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, cons
                            nullptr, nullptr, p->lse_out);
   }
   if (p->mode == MSA_MODE_DECODE) {
+    if (p->lse_out) return fail(MSA_ERR_UNSUPPORTED, "lse_out is written by prefill only (pass NULL for decode)");
     if (p->lmax < 1 || p->lmax > kMaxN) return fail(MSA_ERR_INVALID_ARG, "lmax=%lld out of range", (long long)p->lmax);
     if ((s = check_ptr(p->seqlens, "seqlens")) != MSA_OK) return s;
     const int cpt = p->g * p->d_idx / 32;

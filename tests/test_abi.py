@@ -89,6 +89,29 @@ def test_forward_param_validation(lib):
                       seqlens=None, query_chunk=0)
     assert lib.msa_forward_workspace(ctypes.byref(d)) > 0
     assert lib.msa_forward(ctypes.byref(d), P, P, P, P, P, None, P, P, 1 << 40, None) == 1   # seqlens NULL
+    d.lse_out = P
+    assert lib.msa_forward(ctypes.byref(d), P, P, P, P, P, None, P, P, 1 << 40, None) == 2   # lse: prefill only
+    p = msa.prefill_params(1000, 8, 2, 64, 32, 4)
+    p.lse_out = P + 4                                                                       # unaligned
+    assert lib.msa_forward(ctypes.byref(p), P, P, P, P, P, None, P, P, 1 << 40, None) == 1
+
+
+def test_index_kl_validation_without_cuda(lib):
+    """msa_index_kl checks its shapes and pointers before anything is enqueued: prefill shapes,
+    at most 8 heads per group, the Main Branch's sequence limit, a workspace large enough."""
+    P = 1 << 12
+    p = msa.prefill_params(3000, 16, 2, 128, 64, 8)
+    need = lib.msa_index_kl_workspace(ctypes.byref(p))
+    assert need > 0
+    assert lib.msa_index_kl(ctypes.byref(p), P, P, P, P, P, P, 0.0, P, P, need - 1, None) == 3
+    assert lib.msa_index_kl(ctypes.byref(p), P, P, P, P, P, None, 0.0, P, P, need, None) == 1   # lse NULL
+    assert lib.msa_index_kl(ctypes.byref(p), P, P, P, P, P, P, -1.0, P, P, need, None) == 1     # idx_scale
+    r16 = msa.prefill_params(3000, 32, 2, 128, 64, 8)                                          # 16 heads per group
+    assert lib.msa_index_kl_workspace(ctypes.byref(r16)) == 0
+    assert lib.msa_index_kl(ctypes.byref(r16), P, P, P, P, P, P, 0.0, P, P, 1 << 40, None) == 2
+    dec = msa.MsaParams(mode=1, hq=16, g=2, d=128, d_idx=64, bk=128, k=8, scale=0.0, n=4, lmax=1000,
+                        seqlens=P, query_chunk=0)
+    assert lib.msa_index_kl(ctypes.byref(dec), P, P, P, P, P, P, 0.0, P, P, 1 << 40, None) == 2
 
 
 def test_forward_host_validation_without_cuda(lib):
