@@ -71,39 +71,50 @@ __device__ __forceinline__ CsrChunk csr_chunk(const CsrParams& P, int c) {
 // The ids of a row are accepted when they are -1 padded at the end, strictly
 // ascending, and each lies in [0, bl]. Otherwise the row is dropped (no output) and
 // MSA_ERR_DEVICE_BOUNDS is recorded.
-__device__ __forceinline__ bool csr_row_valid(const int32_t* ids, int k, int bl) {
+// (Loops over the 32 possible slots are unrolled with the row's k as a predicate, so the
+// ids stay in registers.)
+__device__ __forceinline__ bool csr_row_valid(const int32_t (&ids)[32], int k, int bl) {
   int prev = -1;
-  bool ended = false;
-  for (int s = 0; s < k; ++s) {
-    const int b = ids[s];
-    if (b < 0) {
-      if (b != -1) return false;
-      ended = true;
-      continue;
+  bool ended = false, ok = true;
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+    if (s < k) {
+      const int b = ids[s];
+      if (b < 0) {
+        ok = ok && (b == -1);
+        ended = true;
+      } else {
+        ok = ok && !ended && b > prev && b <= bl;
+        prev = b;
+      }
     }
-    if (ended || b <= prev || b > bl) return false;
-    prev = b;
   }
-  return true;
+  return ok;
 }
 
 // builds the membership masks of query tile t for group g into smem bm[nbv * 4], nbv the
 // blocks tile t can see
 __device__ __forceinline__ void csr_build_masks(const CsrParams& P, int t, int nbv, int g, uint32_t* bm,
-                                                int32_t* my_ids, bool& row_ok) {
+                                                int32_t (&my_ids)[32], bool& row_ok) {
   const int r = threadIdx.x;
   for (int w = r; w < nbv * 4; w += blockDim.x) bm[w] = 0u;
   __syncthreads();
   const int64_t i = static_cast<int64_t>(t) * 128 + r;
   row_ok = false;
+#pragma unroll
+  for (int s = 0; s < 32; ++s) my_ids[s] = -1;
   if (i < P.N) {
     const int32_t* src = P.block_ids + (i * P.G + g) * P.k;
-    for (int s = 0; s < P.k; ++s) my_ids[s] = src[s];
+#pragma unroll
+    for (int s = 0; s < 32; ++s)
+      if (s < P.k) my_ids[s] = src[s];
     row_ok = csr_row_valid(my_ids, P.k, static_cast<int>(i / P.bk));
     if (!row_ok) record_error(MSA_ERR_DEVICE_BOUNDS, kKidCsr);
-    if (row_ok)
-      for (int s = 0; s < P.k; ++s)
-        if (my_ids[s] >= 0) atomicOr(&bm[my_ids[s] * 4 + (r >> 5)], 1u << (r & 31));
+    if (row_ok) {
+#pragma unroll
+      for (int s = 0; s < 32; ++s)
+        if (s < P.k && my_ids[s] >= 0) atomicOr(&bm[my_ids[s] * 4 + (r >> 5)], 1u << (r & 31));
+    }
   }
   __syncthreads();
 }
@@ -237,15 +248,25 @@ __global__ void __launch_bounds__(128) csr_scatter_kernel(const __grid_constant_
   const uint32_t* hist = P.hist + T.hist[c];
   const uint32_t* bstart = P.bucket_start + T.bucket[c] + c;
   int32_t* entries = P.entries + T.entry[c];
-  for (int s = 0; s < P.k; ++s) {
-    const int b = ids[s];
-    if (b < 0) break;
-    const uint32_t* m = bm + b * 4;
-    uint32_t rank = __popc(m[r >> 5] & below);
-    for (int w = 0; w < (r >> 5); ++w) rank += __popc(m[w]);
-    const int64_t bucket = static_cast<int64_t>(g) * ch.nbk + b;
-    const uint32_t pos = bstart[bucket] + hist[bucket * ch.nt + qt] + rank;
-    entries[pos] = static_cast<int32_t>((i << 5) | s);
+  // the bucket starts and tile offsets of all of the row's slots are loaded before any is
+  // used (one memory round trip), then each slot's entry goes to its place
+  uint32_t base[32];
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+    base[s] = 0u;
+    if (s < P.k && ids[s] >= 0) {
+      const int64_t bucket = static_cast<int64_t>(g) * ch.nbk + ids[s];
+      base[s] = __ldg(bstart + bucket) + __ldg(hist + bucket * ch.nt + qt);
+    }
+  }
+#pragma unroll
+  for (int s = 0; s < 32; ++s) {
+    if (s < P.k && ids[s] >= 0) {
+      const uint32_t* m = bm + ids[s] * 4;
+      uint32_t rank = __popc(m[r >> 5] & below);
+      for (int w = 0; w < (r >> 5); ++w) rank += __popc(m[w]);
+      entries[base[s] + rank] = static_cast<int32_t>((i << 5) | s);
+    }
   }
 }
 

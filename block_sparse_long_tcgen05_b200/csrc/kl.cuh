@@ -170,9 +170,12 @@ kl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
           // the query's index row, RP copies (one per row of the query's 8-row group)
           const uint4* src = reinterpret_cast<const uint4*>(P.q_idx + ((static_cast<int64_t>(e >> 5) * P.G + g) * DI));
           uint8_t* grp = smem + C::kQiOff + qs * C::kITileBytes + lane * C::kIGroupBytes;
+          uint4 row[DI / 8];                                     // the whole row in flight at once
+#pragma unroll
+          for (int ch = 0; ch < DI / 8; ++ch) row[ch] = __ldg(src + ch);
 #pragma unroll
           for (int ch = 0; ch < DI / 8; ++ch) {                  // 16-byte chunks of the row
-            const uint4 v = __ldg(src + ch);
+            const uint4 v = row[ch];
             const int pnl = (ch * 16) / C::kIRowBytes;
             const int cin = ((ch * 16) % C::kIRowBytes) / 16;    // chunk within the panel row
 #pragma unroll
