@@ -29,7 +29,8 @@
 //               once every product of the current item has completed)
 //   warp 1      tcgen05.mma issue of S and Y, in tile order
 //   warp 2      query gather: TMA boxes of q as in the KV-outer pass; the index rows by
-//               16-byte loads, written RP times into the swizzled Qi tile
+//               16-byte loads, written RP times into the swizzled Qi tile (one query per
+//               store instruction, so the lanes' stores fall into distinct banks)
 //   warp 3      idle
 //   warps 4-11  two reduction warpgroups; tile n goes to warpgroup n % 2
 #pragma once
@@ -164,24 +165,37 @@ kl_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUte
         if (!w_ok) { ok = false; break; }
         if (lane == 0) mbar_arrive_expect_tx(&q_full[qs], nq * RP * 128 * C::kPanels);
         __syncwarp();
-        if (lane < nq) {
+        if (lane < nq)
           tma_load_4d(smem + C::kQOff + qs * C::kTileBytes + lane * C::kGroupBytes, &tm_q, &q_full[qs], 0, g * P.R, 0,
                       e >> 5);
-          // the query's index row, RP copies (one per row of the query's 8-row group)
-          const uint4* src = reinterpret_cast<const uint4*>(P.q_idx + ((static_cast<int64_t>(e >> 5) * P.G + g) * DI));
-          uint8_t* grp = smem + C::kQiOff + qs * C::kITileBytes + lane * C::kIGroupBytes;
-          uint4 row[DI / 8];                                     // the whole row in flight at once
+        {
+          // Each query's index row, RP copies (one per row of the query's 8-row group). The whole
+          // warp writes one query at a time: lane l takes 16-byte chunk l % CPR of the row into
+          // rows (l / CPR) + t * (32 / CPR), so the lanes of one store hit distinct banks.
+          constexpr int CPR = DI / 8;                 // 16-byte chunks per row
+          constexpr int RPI = 32 / CPR;               // rows written per store instruction
+          const int ch = lane % CPR, rsub = lane / CPR;
+          const int pnl = (ch * 16) / C::kIRowBytes;
+          const int cin = ((ch * 16) % C::kIRowBytes) / 16;
+          uint4 row[TQ];                              // chunk ch of every query's row, loads in flight together
 #pragma unroll
-          for (int ch = 0; ch < DI / 8; ++ch) row[ch] = __ldg(src + ch);
+          for (int qq = 0; qq < TQ; ++qq) {
+            const int eq = __shfl_sync(0xffffffffu, e, qq);
+            row[qq] = (qq < nq) ? __ldg(reinterpret_cast<const uint4*>(
+                                       P.q_idx + (static_cast<int64_t>(eq >> 5) * P.G + g) * DI) + ch)
+                                : make_uint4(0u, 0u, 0u, 0u);
+          }
+          uint8_t* tile = smem + C::kQiOff + qs * C::kITileBytes;
 #pragma unroll
-          for (int ch = 0; ch < DI / 8; ++ch) {                  // 16-byte chunks of the row
-            const uint4 v = row[ch];
-            const int pnl = (ch * 16) / C::kIRowBytes;
-            const int cin = ((ch * 16) % C::kIRowBytes) / 16;    // chunk within the panel row
+          for (int qq = 0; qq < TQ; ++qq) {
+            if (qq < nq) {
+              uint8_t* grp = tile + qq * C::kIGroupBytes + pnl * C::kIAtom;
 #pragma unroll
-            for (int r = 0; r < 8; ++r) {
-              const int sw = C::kISw64 ? (cin ^ ((r >> 1) & 3)) : (cin ^ r);
-              st_shared_v4(smem_u32(grp + pnl * C::kIAtom + r * C::kIRowBytes + sw * 16), v.x, v.y, v.z, v.w);
+              for (int t = 0; t < RP / RPI; ++t) {
+                const int r = rsub + t * RPI;
+                const int sw = C::kISw64 ? (cin ^ ((r >> 1) & 3)) : (cin ^ r);
+                st_shared_v4(smem_u32(grp + r * C::kIRowBytes + sw * 16), row[qq].x, row[qq].y, row[qq].z, row[qq].w);
+              }
             }
           }
           fence_proxy_async_smem();
