@@ -31,6 +31,8 @@ def _close(a, ref, atol, rtol, what):
     (2500 + 77, 16, 4, 128, 64, 8, 64, None),
     (1800, 8, 2, 64, 128, 16, 32, None),
     (4200, 64, 8, 128, 128, 16, 128, 160),         # the workload dims (R = 8), sampled rows
+    (1500, 2, 2, 64, 64, 8, 128, None),            # one head per group (R = 1)
+    (1300 + 5, 4, 2, 128, 32, 4, 64, None),        # R = 2
 ])
 def test_index_kl_matches_oracle(cuda_ok, N, Hq, G, d, d_idx, k, Bk, rows):
     cfg = synth.PrefillConfig("t", N=N, Hq=Hq, G=G, d=d, d_idx=d_idx, k=k, idx_range=3 if d_idx == 32 else 4,
