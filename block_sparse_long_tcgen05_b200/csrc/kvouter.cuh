@@ -17,19 +17,23 @@
 //   the unnormalised O (bf16) and (m, l) go to the query's slot s; a later pass merges
 //   the k slots of every query (no atomics).
 //
-// Roles (4 + 4 * kKvSoftmaxWGs + 4 warps; 16 with two softmax warpgroups):
-//   warp 0        TMA loads of K_b and V_b (two buffers each: the next item's block loads
-//                 while the current one is still in use)
+// Roles (16 warps):
+//   warp 0        TMA loads of K_b and V_b into a ring of three block slots (K of item i,
+//                 V of item i, K of item i + 1, ...): a slot is refilled once the product
+//                 that read its previous block has completed
 //   warp 1        tcgen05.mma issue of S = Q K^T, in tile order
 //   warp 2        TMA gather of query rows (one 2 KB box per 8 rows: both 64-column panels)
 //   warp 3        tcgen05.mma issue of O = P V, in tile order. Two issuers, because an issue
 //                 sequence stalls while the tensor pipe is busy: a PV that is ready does not
 //                 wait behind the S product of the next tile, nor the other way round.
-//   softmax       kKvSoftmaxWGs warpgroups from warp 4 on; tile n goes to warpgroup
-//                 n % kKvSoftmaxWGs, which takes S(n) from TMEM region n % kKvSoftmaxWGs and
-//                 writes P over it; the warpgroups take turns on the exp unit
-//   epilogue      the last warpgroup: O from TMEM to bf16 staging, TMA-stored per query
-// TMEM: S/P regions at columns 128 * w, w < kKvSoftmaxWGs; O region(s) after them.
+//   softmax       two warpgroups (warps 4-11); tile n goes to warpgroup n % 2 and to TMEM
+//                 S/P region n % 3. With three regions for two warpgroups, S(n + 2) needs
+//                 only PV(n - 1) to be done, so it is computed while the warpgroup still
+//                 works on tile n, and the warpgroup goes from one tile to its next
+//                 without waiting for its own PV and S products.
+//   epilogue      warps 12-15: O from TMEM to bf16 staging, TMA-stored per query
+// TMEM: S/P regions at columns 0, 128 and 256; O (one buffer: the epilogue reads it out
+// while the next tile's softmax runs) at column 384.
 //
 // Shared-memory layouts (all 128-byte swizzled, 1024-byte aligned):
 //   K, V: [panel][BK keys][128 B]                      (8-row group stride 1 KB, panel BK * 128 B)
@@ -40,18 +44,12 @@
 namespace msa {
 
 constexpr int kKvItemTiles = 4;
-constexpr int kKvQStages = 2;
-// Softmax warpgroups = S/P regions of TMEM (128 columns each). Tile n goes to warpgroup
-// n % kKvSoftmaxWGs. Two (the default): O is double-buffered and every thread may hold 128
-// registers. Three: a warpgroup's next tile can start its S product while the other two run
-// their softmax, O (128 columns) is single-buffered, and the 640 threads get 96 registers
-// each (measured slower at d = 128: the softmax then spills).
-#ifndef MSA_KV_SOFTMAX_WGS
-#define MSA_KV_SOFTMAX_WGS 2
-#endif
-constexpr int kKvSoftmaxWGs = MSA_KV_SOFTMAX_WGS;
-constexpr int kKvOBufs = (kKvSoftmaxWGs == 2) ? 2 : 1;
-static_assert(kKvSoftmaxWGs * 128 + kKvOBufs * 128 <= 512, "TMEM holds 512 columns");
+constexpr int kKvQStages = 3;      // query tiles in shared memory
+constexpr int kKvSlots = 3;        // K / V block slots in shared memory
+constexpr int kKvSoftmaxWGs = 2;   // softmax warpgroups; tile n goes to n % 2
+constexpr int kKvSRegions = 3;     // S/P regions of TMEM (128 columns each); tile n uses n % 3
+constexpr int kKvOCol = kKvSRegions * 128;   // the O accumulator (128 columns)
+static_assert(kKvOCol + 128 <= 512, "TMEM holds 512 columns");
 constexpr int kKvEpiWarp = 4 + 4 * kKvSoftmaxWGs;   // first warp of the epilogue warpgroup
 constexpr int kKvThreads = 32 * (kKvEpiWarp + 4);
 
@@ -63,9 +61,8 @@ struct KvCfg {
   static constexpr int kKvPanel = BK * 128;              // one 64-column panel of a K or V block
   static constexpr int kGroupBytes = kPanels * 1024;     // one 8-row group, all panels
   static constexpr int TQ = 128 / RP;
-  static constexpr int kKOff = 0;                        // 2 K buffers
-  static constexpr int kVOff = 2 * kKvBytes;             // 2 V buffers
-  static constexpr int kQOff = 4 * kKvBytes;             // kKvQStages query stages
+  static constexpr int kKvOff = 0;                       // kKvSlots K / V block slots
+  static constexpr int kQOff = kKvSlots * kKvBytes;      // kKvQStages query stages
   static constexpr int kStgOff = kQOff + kKvQStages * kTileBytes;   // O staging (one tile)
   static constexpr int kBarOff = kStgOff + kTileBytes;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;
@@ -99,19 +96,20 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-  uint64_t* k_full = bars + 0;              // [2] per K buffer
-  uint64_t* k_empty = bars + 2;             // [2]
-  uint64_t* v_full = bars + 4;              // [2] per V buffer
-  uint64_t* v_empty = bars + 6;             // [2]
-  uint64_t* q_full = bars + 8;              // [QS]
-  uint64_t* q_empty = bars + 8 + QS;        // [QS]
-  constexpr int NB = kKvSoftmaxWGs, NO = kKvOBufs;
-  uint64_t* s_full = bars + 8 + 2 * QS;     // [NB] S of tile n in TMEM (S issuer -> softmax)
-  uint64_t* p_full = s_full + NB;           // [NB] P written over S (softmax, 4 warps -> PV issuer)
-  uint64_t* sp_free = p_full + NB;          // [NB] PV done: S/P region free (PV issuer -> S issuer)
-  uint64_t* o_full = sp_free + NB;          // [NO] PV done (PV issuer -> epilogue)
-  uint64_t* o_free = o_full + NO;           // [NO] O read out (epilogue, 4 warps -> PV issuer)
-  uint64_t* s_done = o_free + NO;           // all S products of the CTA complete
+  constexpr int NS = kKvSRegions, NW = kKvSoftmaxWGs, KS = kKvSlots;
+  // a slot's loads alternate between K and V blocks, read by different issuers; each issuer
+  // waits on its own full barrier, so that it sees every phase of it
+  uint64_t* k_full = bars + 0;              // [KS] K block landed in slot s (producer -> S issuer)
+  uint64_t* v_full = k_full + KS;           // [KS] V block landed in slot s (producer -> PV issuer)
+  uint64_t* kv_empty = v_full + KS;         // [KS] slot s read out (either issuer -> producer)
+  uint64_t* q_full = kv_empty + KS;         // [QS]
+  uint64_t* q_empty = q_full + QS;          // [QS]
+  uint64_t* s_full = q_empty + QS;          // [NS] S of tile n in TMEM (S issuer -> softmax)
+  uint64_t* p_full = s_full + NS;           // [NS] P written over S (softmax, 4 warps -> PV issuer)
+  uint64_t* sp_free = p_full + NS;          // [NS] PV done: S/P region free (PV issuer -> S issuer)
+  uint64_t* o_full = sp_free + NS;          // PV done (PV issuer -> epilogue)
+  uint64_t* o_free = o_full + 1;            // O read out (epilogue, 4 warps -> PV issuer)
+  uint64_t* s_done = o_free + 1;            // all S products of the CTA complete
   uint64_t* pv_done = s_done + 1;           // all PV products of the CTA complete
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 1);
   WaitCtl* abort_flag = reinterpret_cast<WaitCtl*>(tmem_slot + 2);
@@ -120,12 +118,11 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1);
-    }
+    for (int i = 0; i < KS; ++i) { mbar_init(&k_full[i], 1); mbar_init(&v_full[i], 1); mbar_init(&kv_empty[i], 1); }
     for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
-    for (int i = 0; i < NB; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4); mbar_init(&sp_free[i], 1); }
-    for (int i = 0; i < NO; ++i) { mbar_init(&o_full[i], 1); mbar_init(&o_free[i], 4); }
+    for (int i = 0; i < NS; ++i) { mbar_init(&s_full[i], 1); mbar_init(&p_full[i], 4); mbar_init(&sp_free[i], 1); }
+    mbar_init(o_full, 1);
+    mbar_init(o_free, 4);
     mbar_init(s_done, 1);
     mbar_init(pv_done, 1);
     wait_ctl_init(abort_flag);
@@ -145,34 +142,37 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
   if (warp == 0) {
     // ------------------------------ K / V producer ------------------------------
-    // Item ni uses K / V buffer ni % 2; a buffer is refilled once the last S (for K) or
-    // PV (for V) product of the item before the previous one has completed.
+    // Load j (K of item i is j = 2i, its V j = 2i + 1) goes to slot j % 3, once the product
+    // that read load j - 3 has completed: the last PV of item i - 2 (for K of item i) or the
+    // last S of item i - 1 (for V of item i).
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int ni = 0, kn = 0, vn = 0;
+      int j = 0;
+      bool ok = true;
       int4 nxt = first_item;
-      for (int t = blockIdx.x; t < n_items; t += grid, ++ni) {
+      for (int t = blockIdx.x; t < n_items && ok; t += grid) {
         const int4 it = nxt;
         if (t + grid < n_items) nxt = P.items[t + grid];
         const int g = it.x / P.nbk, b = it.x % P.nbk;
-        const int kb = ni & 1;
-        const uint32_t ph = static_cast<uint32_t>(ni >> 1) & 1;
-        if (!mbar_wait(&k_empty[kb], ph ^ 1, abort_flag, kKidKvOuter)) break;
-        mbar_arrive_expect_tx(&k_full[kb], C::kKvBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(smem + C::kKOff + kb * C::kKvBytes + p * C::kKvPanel, &tm_k, &k_full[kb], p * 64, g, b * BK);
-        ++kn;
-        if (!mbar_wait(&v_empty[kb], ph ^ 1, abort_flag, kKidKvOuter)) break;
-        mbar_arrive_expect_tx(&v_full[kb], C::kKvBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(smem + C::kVOff + kb * C::kKvBytes + p * C::kKvPanel, &tm_v, &v_full[kb], p * 64, g, b * BK);
-        ++vn;
+        for (int kv = 0; kv < 2; ++kv, ++j) {
+          const int sl = j % KS;
+          const uint32_t ph = static_cast<uint32_t>(j / KS) & 1;
+          if (!mbar_wait(&kv_empty[sl], ph ^ 1, abort_flag, kKidKvOuter)) { ok = false; break; }
+          uint64_t* full = kv ? &v_full[sl] : &k_full[sl];
+          mbar_arrive_expect_tx(full, C::kKvBytes);
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_3d(smem + C::kKvOff + sl * C::kKvBytes + p * C::kKvPanel, kv ? &tm_v : &tm_k, full, p * 64, g,
+                        b * BK);
+        }
       }
-      // drain: the last K and V loads issued into each buffer must land before the CTA exits
-      for (int x = 1; x <= 2; ++x) {
-        if (kn >= x) mbar_wait(&k_full[(kn - x) & 1], static_cast<uint32_t>((kn - x) >> 1) & 1, nullptr, kKidKvOuter);
-        if (vn >= x) mbar_wait(&v_full[(vn - x) & 1], static_cast<uint32_t>((vn - x) >> 1) & 1, nullptr, kKidKvOuter);
+      // drain: the last load issued into each slot must land before the CTA exits (load L is
+      // phase (L / 2) / 3 of its slot's K or V barrier)
+      for (int x = 1; x <= KS; ++x) {
+        const int L = j - x;
+        if (L >= 0)
+          mbar_wait((L & 1) ? &v_full[L % KS] : &k_full[L % KS], static_cast<uint32_t>((L >> 1) / KS) & 1, nullptr,
+                    kKidKvOuter);
       }
     }
   } else if (warp == 2) {
@@ -220,10 +220,10 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------ MMA issuers ------------------------------
-    // warp 1: S(n) once its query rows and its item's K are in shared memory and PV(n - NB),
+    // warp 1: S(n) once its query rows and its item's K are in shared memory and PV(n - 3),
     //         which read P from the same TMEM columns, has completed.
     // warp 3: PV(n) once P(n) is written, its item's V is in shared memory and the epilogue
-    //         has read O(n - NO) out of the same TMEM columns.
+    //         has read O(n - 1) out of TMEM.
     if (lane == 0) {
       const bool is_s = (warp == 1);
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, BK, false);
@@ -235,16 +235,16 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int4 it = nxt;
         if (t + grid < n_items) nxt = P.items[t + grid];
         const int ntiles = (it.z + TQ - 1) / TQ;
-        const int kb = ni & 1;
-        const uint32_t ph = static_cast<uint32_t>(ni >> 1) & 1;
-        const uint32_t k_addr = smem_u32(smem + C::kKOff + kb * C::kKvBytes);
-        const uint32_t v_addr = smem_u32(smem + C::kVOff + kb * C::kKvBytes);
-        if (!mbar_wait(is_s ? &k_full[kb] : &v_full[kb], ph, abort_flag, kKidKvOuter)) { ok = false; break; }
+        const int sl = (2 * ni + (is_s ? 0 : 1)) % KS;            // slot of this item's K or V
+        const uint32_t kv_addr = smem_u32(smem + C::kKvOff + sl * C::kKvBytes);
+        // item ni's K (V) is the (ni / 3)-th K (V) block of its slot
+        if (!mbar_wait(is_s ? &k_full[sl] : &v_full[sl], static_cast<uint32_t>(ni / KS) & 1, abort_flag, kKidKvOuter)) {
+          ok = false;
+          break;
+        }
         for (int j = 0; j < ntiles; ++j, ++n) {
-          const int w = n % NB;                                   // S/P region and warpgroup
-          const uint32_t u = static_cast<uint32_t>(n / NB) & 1;   // phase parity of region w
-          const int ob = n % NO;                                  // O region
-          const uint32_t uo = static_cast<uint32_t>(n / NO) & 1;
+          const int w = n % NS;                                   // S/P region
+          const uint32_t u = static_cast<uint32_t>(n / NS) & 1;   // phase parity of region w
           if (is_s) {
             const int qs = n % QS;
             if (!mbar_wait(&q_full[qs], static_cast<uint32_t>(n / QS) & 1, abort_flag, kKidKvOuter) ||
@@ -259,28 +259,28 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int kk = 0; kk < D / 16; ++kk) {
               const uint64_t adesc =
                   smem_desc(q_addr + (kk >> 2) * 1024 + (kk & 3) * 32, 16, C::kGroupBytes, kLayoutSw128);
-              const uint64_t bdesc = smem_desc(k_addr + (kk >> 2) * C::kKvPanel + (kk & 3) * 32, 16, 1024, kLayoutSw128);
+              const uint64_t bdesc = smem_desc(kv_addr + (kk >> 2) * C::kKvPanel + (kk & 3) * 32, 16, 1024, kLayoutSw128);
               umma_bf16(d_s, adesc, bdesc, idesc_s, kk > 0);
             }
             umma_commit(&q_empty[qs]);
             umma_commit(&s_full[w]);
-            if (j == ntiles - 1) umma_commit(&k_empty[kb]);
+            if (j == ntiles - 1) umma_commit(&kv_empty[sl]);
           } else {
             if (!mbar_wait(&p_full[w], u, abort_flag, kKidKvOuter) ||
-                !mbar_wait(&o_free[ob], uo ^ 1, abort_flag, kKidKvOuter)) {
+                !mbar_wait(o_free, (static_cast<uint32_t>(n) & 1) ^ 1, abort_flag, kKidKvOuter)) {
               ok = false;
               break;
             }
             tc_fence_after();
-            const uint32_t d_o = tmem + NB * 128 + ob * 128;
+            const uint32_t d_o = tmem + kKvOCol;
             const uint32_t a_p = tmem + w * 128;
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-              umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(v_addr + kk * 2048, C::kKvPanel, 1024, kLayoutSw128), idesc_o,
+              umma_bf16_ts(d_o, a_p + kk * 8, smem_desc(kv_addr + kk * 2048, C::kKvPanel, 1024, kLayoutSw128), idesc_o,
                            kk > 0);
             umma_commit(&sp_free[w]);
-            umma_commit(&o_full[ob]);
-            if (j == ntiles - 1) umma_commit(&v_empty[kb]);
+            umma_commit(o_full);
+            if (j == ntiles - 1) umma_commit(&kv_empty[sl]);
           }
         }
       }
@@ -312,14 +312,12 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int g = it.x / P.nbk;
       const int ntiles = (it.z + TQ - 1) / TQ;
       for (int j = 0; j < ntiles; ++j, ++nt) {
-        const int ob = nt % NO;
-        const uint32_t uo = static_cast<uint32_t>(nt / NO) & 1;
         const int nq = min(TQ, it.z - j * TQ);
         const int qw = quad * QPW + lane;         // the query whose stores this lane issues
         const bool st_lane = (lane < QPW) && (qw < nq);
         const int e = st_lane ? __ldg(P.entries + it.y + j * TQ + qw) : 0;
-        const uint32_t t_o = tmem + lane_base + NB * 128 + ob * 128;
-        if (!mbar_wait(&o_full[ob], uo, abort_flag, kKidKvOuter)) { fail = true; break; }
+        const uint32_t t_o = tmem + lane_base + kKvOCol;
+        if (!mbar_wait(o_full, static_cast<uint32_t>(nt) & 1, abort_flag, kKidKvOuter)) { fail = true; break; }
         tc_fence_after();
         if (lane < QPW) bulk_wait_read_all();     // previous tile's stores have read the rows
         __syncwarp();
@@ -331,7 +329,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           if (c == D / 32 - 1) {
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&o_free[ob]);
+            if (lane == 0) mbar_arrive(o_free);
           }
 #pragma unroll
           for (int x = 0; x < 4; ++x) {              // four 16-byte chunks of 8 columns
@@ -367,11 +365,11 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     // ------------------------------ softmax warpgroups ------------------------------
     // The four warps of a warpgroup never wait for one another: each hands its rows over
     // through mbarrier arrivals (P to the PV issuer).
-    const int wg = (warp - 4) >> 2;               // takes tiles with nt % NB == wg
+    const int wg = (warp - 4) >> 2;               // takes tiles with nt % NW == wg
     const int quad = warp & 3;
     const int m = quad * 32 + lane;               // row of the tile == TMEM lane
     const int q = m / RP, r = m % RP;
-    const uint32_t t_s = tmem + (static_cast<uint32_t>(quad * 32) << 16) + wg * 128;
+    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
     int nt = 0;
     bool fail = false;
     int e_pref = 0, pref_nt = -1;   // CSR entry of this thread's row in the warpgroup's next tile
@@ -382,8 +380,10 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const int g = it.x / P.nbk, b = it.x % P.nbk;
       const int ntiles = (it.z + TQ - 1) / TQ;
       for (int j = 0; j < ntiles; ++j, ++nt) {
-        if (nt % NB != wg) continue;
-        const uint32_t u = static_cast<uint32_t>(nt / NB);
+        if (nt % NW != wg) continue;
+        const int sr = nt % NS;                     // S/P region of this tile
+        const uint32_t u = static_cast<uint32_t>(nt / NS);
+        const uint32_t t_s = t_lane + sr * 128;
         const int nq = min(TQ, it.z - j * TQ);
         const bool valid = (q < nq) && (r < P.R);
         const int e = (pref_nt == nt) ? e_pref : (valid ? __ldg(P.entries + it.y + j * TQ + q) : 0);
@@ -392,21 +392,21 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // load the entry for this warpgroup's next tile now (same item or the next one); rows
         // past that tile's queries read a neighbouring entry that is never used
         {
-          int jn = j + NB;
+          int jn = j + NW;
           const int32_t* base = nullptr;
           if (jn < ntiles) {
             base = P.entries + it.y;
           } else if (t + grid < n_items && (jn -= ntiles) < (nxt.z + TQ - 1) / TQ) {
             base = P.entries + nxt.y;
           }
-          pref_nt = base ? nt + NB : -1;
+          pref_nt = base ? nt + NW : -1;
           if (base) e_pref = __ldg(base + jn * TQ + q);
         }
         const int limit = !valid ? -1 : ((b == i / BK) ? (i % BK) : BK - 1);   // keys c <= limit are visible
         // warps whose rows all see the whole block skip the per-key mask
         const bool whole = __all_sync(0xffffffffu, limit == BK - 1);
         // ---- row max (pass 1 over S; two 32-column loads per TMEM wait, 4 independent chains)
-        if (!mbar_wait(&s_full[wg], u & 1, abort_flag, kKidKvOuter)) { fail = true; break; }
+        if (!mbar_wait(&s_full[sr], u & 1, abort_flag, kKidKvOuter)) { fail = true; break; }
         tc_fence_after();
         float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
         constexpr int LPW = (NCH >= 2) ? 2 : 1;   // 32-column loads per TMEM wait
@@ -467,7 +467,7 @@ kvouter_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[wg]);
+        if (lane == 0) mbar_arrive(&p_full[sr]);
         if (valid) {
           const int64_t il = static_cast<int64_t>(i) - P.row0;
           P.ml[((il * P.G + g) * P.k + s) * P.R + r] = make_float2(mref, (l4[0] + l4[1]) + (l4[2] + l4[3]));
