@@ -56,6 +56,22 @@ __device__ __forceinline__ IdxTopkItem idx_topk_item(const IdxTopkParams& P, int
   return it;
 }
 
+// Shared memory of the fused kernel: the query tiles of kTopkQBufs items (two tiles each),
+// then a ring of kTopkStages key tiles. One item buffer: an item runs over up to N / 128 key
+// tiles, so loading the next item's queries after the last MMA of the current one costs
+// little, and the freed space deepens the key ring (measured at 128K: 4 stages with one item
+// buffer 14.47-14.49 ms, 5 stages 14.71-14.84, 3 stages with two item buffers 14.70-14.72).
+constexpr int kTopkQBufs = 1;
+constexpr int kTopkStages = 4;
+template <int DI>
+struct IdxTopkCfg {
+  using C = IdxCfg<DI>;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = 2 * kTopkQBufs * C::kTileBytes;
+  static constexpr int kBarOff = kKOff + kTopkStages * C::kTileBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+};
+
 // CTA c's r-th item in snake order, or -1 when the round has none for it
 __device__ __forceinline__ int idx_topk_slot(int r, int total) {
   const int grid = static_cast<int>(gridDim.x);
@@ -68,18 +84,22 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
 index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ IdxTopkParams P) {
   using C = IdxCfg<DI>;
+  using T = IdxTopkCfg<DI>;
+  constexpr int S = kTopkStages, QB = kTopkQBufs;
+  static_assert(QB == 1 || QB == 2, "item buffers");
+  static_assert(T::kSmemBytes <= 227 * 1024, "shared memory");
   static_assert(KM >= 1, "at least one non-local place");
   static_assert(BK == 32 || BK == 64 || BK == 128, "block size");
   constexpr int F = 128 / BK;               // blocks per 128-key tile
   constexpr int kDiag = (F > 1) ? 1 : 0;    // the diagonal key tile holds needed blocks
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::kBarOff);
   uint64_t* q_full = bars + 0;              // [2]
   uint64_t* q_empty = bars + 2;             // [2]
   uint64_t* k_full = bars + 4;              // [stages]
-  uint64_t* k_empty = bars + 4 + kIdxStages;
-  uint64_t* acc_full = bars + 4 + 2 * kIdxStages;   // [2]
+  uint64_t* k_empty = bars + 4 + S;
+  uint64_t* acc_full = bars + 4 + 2 * S;    // [2]
   uint64_t* acc_empty = acc_full + 2;               // [2]
   uint64_t* mma_done = acc_empty + 2;               // [1]
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
@@ -90,7 +110,7 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
-    for (int i = 0; i < kIdxStages; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < S; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 8); }
     mbar_init(mma_done, 1);
     wait_ctl_init(abort_flag);
@@ -120,11 +140,11 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (t < 0) continue;
         const IdxTopkItem it = idx_topk_item(P, t, kDiag);
         if (it.kbend == 0) continue;
-        const int qbuf = n_item & 1;
-        const uint32_t qu = static_cast<uint32_t>(n_item >> 1);
+        const int qbuf = n_item % QB;
+        const uint32_t qu = static_cast<uint32_t>(n_item / QB);
         if (!mbar_wait(&q_empty[qbuf], (qu & 1) ^ 1, abort_flag, kKidIndexScore)) { ok = false; break; }
-        uint8_t* qa_s = smem + C::kQOff + (qbuf * 2 + 0) * C::kTileBytes;
-        uint8_t* qb_s = smem + C::kQOff + (qbuf * 2 + 1) * C::kTileBytes;
+        uint8_t* qa_s = smem + T::kQOff + (qbuf * 2 + 0) * C::kTileBytes;
+        uint8_t* qb_s = smem + T::kQOff + (qbuf * 2 + 1) * C::kTileBytes;
         mbar_arrive_expect_tx(&q_full[qbuf], (it.has_b ? 2 : 1) * C::kTileBytes);
         for (int pnl = 0; pnl < C::kPanels; ++pnl) {
           tma_load_3d(qa_s + pnl * C::kPanelBytes, &tm_q, &q_full[qbuf], pnl * C::kPanelElems, it.g, it.qa * 128);
@@ -134,26 +154,26 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         }
         ++n_item;
         for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
-          const int s = static_cast<int>(ik % kIdxStages);
-          const uint32_t u = static_cast<uint32_t>(ik / kIdxStages);
+          const int s = static_cast<int>(ik % S);
+          const uint32_t u = static_cast<uint32_t>(ik / S);
           if (!mbar_wait(&k_empty[s], (u & 1) ^ 1, abort_flag, kKidIndexScore)) { ok = false; break; }
-          uint8_t* ks = smem + C::kKOff + s * C::kTileBytes;
+          uint8_t* ks = smem + T::kKOff + s * C::kTileBytes;
           mbar_arrive_expect_tx(&k_full[s], C::kTileBytes);
           for (int pnl = 0; pnl < C::kPanels; ++pnl)
             tma_load_3d(ks + pnl * C::kPanelBytes, &tm_k, &k_full[s], pnl * C::kPanelElems, it.g, kb * 128);
         }
       }
       // Drain: every TMA load this thread issued must land before the CTA exits.
-      for (int s = 0; s < kIdxStages; ++s) {
+      for (int s = 0; s < S; ++s) {
         if (ik > s) {
-          const int64_t last = ((ik - 1 - s) / kIdxStages) * kIdxStages + s;
-          mbar_wait(&k_full[s], static_cast<uint32_t>(last / kIdxStages) & 1, nullptr, kKidIndexScore);
+          const int64_t last = ((ik - 1 - s) / S) * S + s;
+          mbar_wait(&k_full[s], static_cast<uint32_t>(last / S) & 1, nullptr, kKidIndexScore);
         }
       }
-      for (int b = 0; b < 2; ++b) {
+      for (int b = 0; b < QB; ++b) {
         if (n_item > b) {
-          const int last = ((n_item - 1 - b) / 2) * 2 + b;
-          mbar_wait(&q_full[b], static_cast<uint32_t>(last >> 1) & 1, nullptr, kKidIndexScore);
+          const int last = ((n_item - 1 - b) / QB) * QB + b;
+          mbar_wait(&q_full[b], static_cast<uint32_t>(last / QB) & 1, nullptr, kKidIndexScore);
         }
       }
     }
@@ -169,22 +189,22 @@ index_topk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (t < 0) continue;
         const IdxTopkItem it = idx_topk_item(P, t, kDiag);
         if (it.kbend == 0) continue;
-        const int qbuf = n_item & 1;
-        const uint32_t qu = static_cast<uint32_t>(n_item >> 1);
+        const int qbuf = n_item % QB;
+        const uint32_t qu = static_cast<uint32_t>(n_item / QB);
         ++n_item;
         if (!mbar_wait(&q_full[qbuf], qu & 1, abort_flag, kKidIndexScore)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t qa_addr = smem_u32(smem + C::kQOff + (qbuf * 2 + 0) * C::kTileBytes);
-        const uint32_t qb_addr = smem_u32(smem + C::kQOff + (qbuf * 2 + 1) * C::kTileBytes);
+        const uint32_t qa_addr = smem_u32(smem + T::kQOff + (qbuf * 2 + 0) * C::kTileBytes);
+        const uint32_t qb_addr = smem_u32(smem + T::kQOff + (qbuf * 2 + 1) * C::kTileBytes);
         for (int kb = 0; kb < it.kbend; ++kb, ++ik) {
-          const int s = static_cast<int>(ik % kIdxStages);
-          const uint32_t u = static_cast<uint32_t>(ik / kIdxStages);
+          const int s = static_cast<int>(ik % S);
+          const uint32_t u = static_cast<uint32_t>(ik / S);
           const int ab = static_cast<int>(ik & 1);
           const uint32_t au = static_cast<uint32_t>(ik >> 1);
           if (!mbar_wait(&k_full[s], u & 1, abort_flag, kKidIndexScore)) { ok = false; break; }
           if (!mbar_wait(&acc_empty[ab], (au & 1) ^ 1, abort_flag, kKidIndexScore)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + C::kKOff + s * C::kTileBytes);
+          const uint32_t k_addr = smem_u32(smem + T::kKOff + s * C::kTileBytes);
           const uint32_t d_a = tmem + ab * 256;
           const uint32_t d_b = d_a + 128;
           const bool a_active = kb < it.qa + kDiag;

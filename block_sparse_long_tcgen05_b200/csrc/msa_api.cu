@@ -408,7 +408,7 @@ size_t index_ws_bytes(int64_t n, int32_t g, int32_t k) {
 template <int DI, int KM, int BK>
 msa_status_t launch_index_topk_km(const CUtensorMap& tq, const CUtensorMap& tk, const IdxTopkParams& P,
                                   cudaStream_t st) {
-  using C = IdxCfg<DI>;
+  using C = IdxTopkCfg<DI>;
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
   std::call_once(once, [] { attr = set_smem(index_topk_kernel<DI, KM, BK>, C::kSmemBytes); });
