@@ -408,12 +408,12 @@ size_t index_ws_bytes(int64_t n, int32_t g, int32_t k) {
 template <int DI, int KM, int BK>
 msa_status_t launch_index_topk_km(const CUtensorMap& tq, const CUtensorMap& tk, const IdxTopkParams& P,
                                   cudaStream_t st) {
-  using C = IdxTopkCfg<DI>;
+  using C = IdxTopkCfg<DI, KM>;
   static std::once_flag once;
   static msa_status_t attr = MSA_OK;
   std::call_once(once, [] { attr = set_smem(index_topk_kernel<DI, KM, BK>, C::kSmemBytes); });
   if (attr != MSA_OK) return attr;
-  const int total = P.G * P.npairs;
+  const int total = P.G * P.nt;
   const int grid = std::min(num_sms(), total);
   ProfScope ps(kPIndexTopk, st);
   index_topk_kernel<DI, KM, BK><<<grid, kIdxThreads, C::kSmemBytes, st>>>(tq, tk, P);
@@ -445,7 +445,6 @@ msa_status_t launch_index_topk(const void* q_idx, const void* k_idx, int64_t n, 
   if ((s = make_map_3d(&tk, k_idx, DI, g, n, DI * 2, row_stride, box0, 1, 128, sw)) != MSA_OK) return s;
   IdxTopkParams P{};
   P.nt = int((n + 127) / 128);
-  P.npairs = (P.nt + 1) / 2;
   P.G = g;
   P.k = k;
   P.N = n;
