@@ -224,6 +224,19 @@ def timed(fn, steps: int, stream) -> float:
     return a.elapsed_time(b) / steps
 
 
+def graph_of(fn) -> "torch.cuda.CUDAGraph":
+    """fn captured once as a CUDA graph (after one call outside the capture, which sets the
+    kernels' attributes); every step of the library is a launch on the caller's stream, so
+    replays run the same kernels on the captured buffers' current contents."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def stage_rates(stages: dict, cfg, peaks: dict) -> dict:
     """Every prefill kernel's achieved rate against its own roofline, from the per-step stage
     times: TFLOP/s of the score and attention products (fraction of the measured bf16 burst
@@ -410,6 +423,14 @@ def run_decode(args, dev, stream, world, rank, peaks, cpu_baseline: bool) -> dic
                         "work_per_launch": scan_bytes,
                         "note": "a read-only stream against a read+write copy peak can read a little above 1"},
            "stages": {k: {"ms_per_step": v[1] / args.steps} for k, v in dstats.items()}}
+    # the same step captured once and replayed as a CUDA graph, as a serving loop would run it
+    g = graph_of(dstep)
+    barrier(world)
+    gms = max_over_ranks(timed(g.replay, args.steps, stream), world)
+    msa.check_device_error(dev)
+    del g
+    out["graph"] = {"ms_per_step": gms, "tokens_per_s": world * dcfg.B / (gms * 1e-3),
+                    "how": "one CUDA graph of the decode step, replayed; CUDA events on the stream"}
     if cpu_baseline:
         seqs = 2
         rate, dt = oracle_decode_rate(dinp, dcfg, seqs)
@@ -438,6 +459,15 @@ def config_report(cfg, dev, stream, args, peaks, rank) -> dict:
     out = {"tokens_per_s": cfg.N / (ms * 1e-3), "ms_per_step": ms, "steps": steps,
            **prefill_rates(rcfg, ms, peaks, 1), "memory_bound": memory_bound_rates(st, rcfg, peaks),
            "stages": {k: round(v["ms_per_step"], 4) for k, v in st.items()}}
+    if cfg.N <= 4096:
+        # launch-bound: the forward captured once as a CUDA graph and replayed
+        from block_sparse_long_tcgen05_b200 import msa
+        g = graph_of(lambda: msa.msa_forward(p, inp["q"], inp["k"], inp["v"], inp["q_idx"], inp["k_idx"],
+                                             o=bufs["o"], block_ids=bufs["ids"], workspace=bufs["ws"]))
+        gms = timed(g.replay, steps, stream)
+        msa.check_device_error(dev)
+        del g
+        out["graph"] = {"ms_per_step": gms, "tokens_per_s": cfg.N / (gms * 1e-3)}
     if not args.no_cpu_baseline:
         rate, dt = oracle_rows_rate(inp, cfg, ORACLE_ROWS.get(cfg.name, 4), seed=11)
         out["cpu_baseline"] = {"value": rate, "unit": "tokens/s", "us_per_query": 1e6 / rate,
