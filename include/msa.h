@@ -165,7 +165,11 @@ MSA_API msa_status_t msa_sparse_attn(const void* q, const void* k, const void* v
  * second and third paragraphs) and takes the stricter of their sequence limits. Decode applies
  * the same definition to the last token of each sequence: one query per sequence cannot fill
  * a KV-stationary tile, so it runs query-stationary, the design the skandtandon.pages.dev note
- * "KV-stationary attention" (The problem) contrasts with the KV-stationary one. */
+ * "KV-stationary attention" (The problem) contrasts with the KV-stationary one.
+ * The call only enqueues kernel launches on `stream` (no host synchronisation, no
+ * allocation) with grids that depend on *p alone (decode: on lmax; the lengths are read on
+ * the device), so it may be captured into a CUDA graph and the graph replayed on new
+ * contents of the same buffers. */
 MSA_API size_t msa_forward_workspace(const msa_params* p);
 MSA_API msa_status_t msa_forward(const msa_params* p, const void* q, const void* k, const void* v, const void* q_idx,
                          const void* k_idx, int32_t* block_ids_out, void* o, void* workspace,
